@@ -1,0 +1,198 @@
+/*
+ * damp.h -- C ABI of libdamp: the decode step of a DAMP-style mixed-precision
+ * recurrent state for Gated DeltaNet (GDN) and Kimi Delta Attention (KDA)
+ * layers, on NVIDIA B200 (sm_100a).
+ *
+ * What the operation is (web pages, cited by title and section):
+ *   - "DAMP: Decay-Aware Mixed-Precision Recurrent-State Quantization",
+ *     arXiv 2608.27513v1 abstract: GDN/KDA recurrent states are FP32 by
+ *     default, their update is memory-bandwidth bound; DAMP keeps high-risk
+ *     channels at higher precision and the rest in INT8 (9.9 bits/value,
+ *     69.1 % less state storage).  The later abstract (mlsanity.com index
+ *     page) names the high-risk *key channels* and FP16, chosen offline under
+ *     a fixed storage budget.
+ *   - "STEPQuant: When and Where Errors Matter in Delta-Rule Recurrent State
+ *     Quantization", Appendix Table C2 (one persistent decode step): (1)
+ *     reconstruct the state from codes and scales or FP16 values, (2)
+ *     X = D S^ + beta k (v^T - k^T D S^) with D = alpha I (GDN) or
+ *     Diag(alpha) (KDA), (3) emit X^T q before requantization, (6) pack codes
+ *     and scales, store the FP16 rows, keeping the old representation valid
+ *     until its readers finish.
+ *
+ * Arithmetic (one reading each where the pages are silent):
+ *   S^_ij   = fp16 value (FP16 row) | fl(code_ij * scale_i) (INT8 row)
+ *   S'_ij   = fl(alpha_i * S^_ij)
+ *   u_j     = sum_i fl(k_i * S'_ij), recursive pairwise order over rows
+ *   delta_j = fl(v_j - u_j);  b_i = fl(beta * k_i)
+ *   X_ij    = fma(b_i, delta_j, S'_ij)           (all of the above in FP32)
+ *   out_j   = sum_i q_i X_ij                     (FP32, from X, any order)
+ *   FP16 rows: X rounded to binary16, nearest-even.
+ *   INT8 rows: a = max_j |X_ij|; scale = fl(a/127); inv = fl(127/a);
+ *              code = nearest integer to the exact X*inv, ties to even.
+ *              a == 0 or inv == +inf -> scale 0, codes 0.
+ *
+ * Conventions for every call:
+ *   - Device memory is owned by the caller (for example allocated by
+ *     PyTorch).  The library allocates no device memory.  The only host
+ *     memory it owns is the damp_pool descriptor.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     that take a stream only enqueue work and return; their results are
+ *     visible after the stream is synchronised.
+ *   - Arguments are checked on the host before anything is enqueued.  A
+ *     negative return means nothing was enqueued (except DAMP_ERR_CUDA, which
+ *     reports a failed enqueue).  Device-side conditions that the host cannot
+ *     see (a slot index out of range, an internal wait that hit its bound)
+ *     set bits in the pool's status word (damp_pool_get_error); kernels never
+ *     trap.
+ *   - Supported shapes: d_k == d_v == d, d in {16, 32, 64, 128}; 1 <= H;
+ *     1 <= n_slots; 0 <= hp_rows <= d_k.
+ *   - Device pointers passed for bulk copies (pool buffer, q, k, v, KDA
+ *     alpha, out, FP32 states) must be 16-byte aligned.
+ */
+#ifndef DAMP_H
+#define DAMP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes --------------------------------------------------------- */
+#define DAMP_OK 0
+#define DAMP_ERR_INVALID_ARGUMENT (-1) /* null pointer, bad enum, bad index map */
+#define DAMP_ERR_UNSUPPORTED (-2)      /* shape outside the supported set       */
+#define DAMP_ERR_MISALIGNED (-3)       /* a pointer is not 16-byte aligned      */
+#define DAMP_ERR_BUFFER_TOO_SMALL (-4) /* buf_bytes < damp_pool_bytes(...)      */
+#define DAMP_ERR_CUDA (-5)             /* a CUDA runtime call failed            */
+
+/* ---- device status word bits (damp_pool_get_error) ----------------------- */
+#define DAMP_EFLAG_SLOT_RANGE 1u /* a slot_idx entry >= n_slots (entry skipped) */
+#define DAMP_EFLAG_TIMEOUT 2u    /* an internal pipeline wait hit its bound     */
+
+/* ---- enums ----------------------------------------------------------------- */
+#define DAMP_FMT_FP32 0     /* plain FP32 state (the pages' unquantized baseline)   */
+#define DAMP_FMT_INT8_ROW 1 /* every row INT8 + FP32 absmax scale (uniform INT8)   */
+#define DAMP_FMT_MIXED 2    /* hp_rows FP16 key rows per head, the rest INT8 (DAMP) */
+
+#define DAMP_GATE_SCALAR 0 /* GDN: alpha is one FP32 per (entry, head)            */
+#define DAMP_GATE_VECTOR 1 /* KDA: alpha is d_k FP32 per (entry, head)            */
+
+#define DAMP_DTYPE_BF16 0 /* q, k, v are bfloat16 */
+#define DAMP_DTYPE_F32 1  /* q, k, v are float32  */
+
+typedef struct damp_pool damp_pool; /* opaque host-side descriptor */
+
+/* Human-readable text of a status code.  Never NULL; static storage. */
+const char* damp_status_string(int status);
+
+/*
+ * Byte layout of one (slot, head) state block.
+ *   *block_bytes  : bytes the format must hold (the algorithmic size:
+ *                   FP32 d_k*d_v*4; quantized 2*hp*d_v + r*d_v + 4*r with
+ *                   r = d_k - hp).  27 FP16 rows at d = 128 give 20,244 B,
+ *                   9.885 bits per value, 69.1 % below FP32 (the pages'
+ *                   "9.9 bits" and "69.1 %", DAMP v1 abstract).
+ *   *block_stride : bytes between consecutive blocks in a pool (block_bytes
+ *                   rounded up to 16 for bulk copies).
+ * Quantized block byte order: r FP32 scales (INT8 rows in increasing key
+ * index) padded to 16 B, then the hp FP16 rows in increasing key index, then
+ * the r INT8 rows in increasing key index.  FP32 blocks: row-major [d_k][d_v].
+ * Either output pointer may be NULL.
+ */
+int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
+                size_t* block_stride);
+
+/*
+ * Bytes the caller must allocate for a pool of n_slots x H blocks: a header
+ * (per-head FP16-row masks and the device status word, 256 B aligned)
+ * followed by the blocks, block (slot, h) at header + (slot*H + h)*stride.
+ */
+int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
+                    size_t* bytes);
+
+/*
+ * Bind a descriptor to a caller-owned device buffer and write its header.
+ *   hp_row_idx : host array [H][hp_rows] of the FP16 key rows of each head
+ *                (the frozen precision map from offline calibration).  Each
+ *                head's entries must be distinct and < d_k; any order.  NULL
+ *                allowed when hp_rows == 0.  Copied; the caller keeps it.
+ *   dev_buf    : device buffer of buf_bytes >= damp_pool_bytes(...), 16-byte
+ *                aligned; stays owned by the caller and must outlive the pool.
+ * The block contents are left as they are (pack them, or restore raw bytes).
+ * Synchronous (writes the header with a blocking copy).  On success *out
+ * receives a descriptor to release with damp_pool_destroy.
+ */
+int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
+                     const uint16_t* hp_row_idx, void* dev_buf, size_t buf_bytes,
+                     damp_pool** out);
+
+/* Release the descriptor (never the caller's device buffer).  NULL is a no-op. */
+int damp_pool_destroy(damp_pool* pool);
+
+/* Byte offset of block (slot, h) from the start of the caller's buffer. */
+int damp_pool_block_offset(const damp_pool* pool, int slot, int h, size_t* offset);
+
+/*
+ * Compress FP32 states into pool slots (prefill hand-off, restore).
+ *   slot_idx : device int32 [n]; entry b < 0 is skipped; >= n_slots sets
+ *              DAMP_EFLAG_SLOT_RANGE and is skipped.
+ *   state    : device float32 [n][H][d_k][d_v].
+ * Entries of slot_idx must be distinct (each block has one writer).
+ */
+int damp_pool_pack(const damp_pool* pool, int n, const int32_t* slot_idx, const float* state,
+                   void* stream);
+
+/*
+ * Reconstruct FP32 states from pool slots (Table C2 step 1: FP16 rows
+ * exactly, INT8 rows as fl(code * scale)).  state: device float32
+ * [n][H][d_k][d_v]; entries with slot_idx < 0 or out of range are zeroed.
+ */
+int damp_pool_unpack(const damp_pool* pool, int n, const int32_t* slot_idx, float* state,
+                     void* stream);
+
+/*
+ * One decode step for every (entry b, head h): read block (slot_idx[b], h),
+ * apply the gated delta rule, write out[b][h][:] = X^T q, requantize the
+ * block in place.
+ *   slot_idx : device int32 [n].  < 0: padding, out row zeroed, block
+ *              untouched.  >= n_slots: DAMP_EFLAG_SLOT_RANGE, out row zeroed.
+ *              Entries must be distinct.
+ *   in_dtype : DAMP_DTYPE_BF16 | DAMP_DTYPE_F32 for q, k, v.
+ *   q, k     : device [n][H][d_k];  v : device [n][H][d_v]  (final values: the
+ *              step applies no scaling or normalisation).
+ *   gate     : DAMP_GATE_SCALAR (alpha device float32 [n][H]) or
+ *              DAMP_GATE_VECTOR (alpha device float32 [n][H][d_k]).
+ *   beta     : device float32 [n][H].
+ *   out      : device float32 [n][H][d_v].
+ * n == 0 is a no-op.  Inputs and out must not alias the pool buffer.
+ */
+int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int in_dtype,
+                     const void* q, const void* k, const void* v, int gate,
+                     const float* alpha, const float* beta, float* out, void* stream);
+
+/*
+ * Read the device status word (DAMP_EFLAG_* bits accumulated since the last
+ * clear) into *flags; clear it when `clear` is non-zero.  Synchronises
+ * `stream`.
+ */
+int damp_pool_get_error(const damp_pool* pool, uint32_t* flags, int clear, void* stream);
+
+/*
+ * Host-only conversion between one raw block (block_stride bytes, as stored
+ * in the pool) of head h and the logical per-row form, rows in key-channel
+ * order: scale[d_k] (0 for FP16 rows), half[d_k][d_v] (binary16 bits, 0 for
+ * INT8 rows), code[d_k][d_v] (0 for FP16 rows); FP32 format: f32[d_k][d_v].
+ * Pointers a format does not use may be NULL.  No CUDA call is made.
+ */
+int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float* scale,
+                          uint16_t* half, int8_t* code, float* f32);
+int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
+                            const uint16_t* half, const int8_t* code, const float* f32,
+                            void* block);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DAMP_H */

@@ -1,0 +1,304 @@
+"""Python binding of libdamp, the B200 decode step of DAMP-style mixed-precision
+recurrent states (Gated DeltaNet / Kimi Delta Attention).
+
+Every function here has the name of the C entry point it marshals arguments
+for (declared in include/damp.h); all work happens in libdamp's CUDA kernels.
+PyTorch supplies device memory and streams only.  Importing this module
+fails if libdamp.so has not been built: there is no fallback path.
+
+Tensor arguments must be contiguous CUDA tensors of the documented dtype;
+``stream`` defaults to the current PyTorch stream of the tensors' device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdamp.so")
+
+DAMP_OK = 0
+DAMP_ERR_INVALID_ARGUMENT = -1
+DAMP_ERR_UNSUPPORTED = -2
+DAMP_ERR_MISALIGNED = -3
+DAMP_ERR_BUFFER_TOO_SMALL = -4
+DAMP_ERR_CUDA = -5
+
+DAMP_EFLAG_SLOT_RANGE = 1
+DAMP_EFLAG_TIMEOUT = 2
+
+DAMP_FMT_FP32 = 0
+DAMP_FMT_INT8_ROW = 1
+DAMP_FMT_MIXED = 2
+DAMP_GATE_SCALAR = 0
+DAMP_GATE_VECTOR = 1
+DAMP_DTYPE_BF16 = 0
+DAMP_DTYPE_F32 = 1
+
+FORMATS = {"fp32": DAMP_FMT_FP32, "int8": DAMP_FMT_INT8_ROW, "mixed": DAMP_FMT_MIXED}
+
+
+class DampError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {damp_status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python -m quantized_linear_attention_damp_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "damp_status_string": (ctypes.c_char_p, [I]),
+        "damp_layout": (I, [I, I, I, I, ctypes.POINTER(S), ctypes.POINTER(S)]),
+        "damp_pool_bytes": (I, [I, I, I, I, I, I, ctypes.POINTER(S)]),
+        "damp_pool_create": (I, [I, I, I, I, I, I, P, P, S, ctypes.POINTER(P)]),
+        "damp_pool_destroy": (I, [P]),
+        "damp_pool_block_offset": (I, [P, I, I, ctypes.POINTER(S)]),
+        "damp_pool_pack": (I, [P, I, P, P, P]),
+        "damp_pool_unpack": (I, [P, I, P, P, P]),
+        "damp_decode_step": (I, [P, I, P, I, P, P, P, I, P, P, P, P]),
+        "damp_pool_get_error": (I, [P, ctypes.POINTER(ctypes.c_uint32), I, P]),
+        "damp_block_to_logical": (I, [P, I, P, P, P, P, P]),
+        "damp_block_from_logical": (I, [P, I, P, P, P, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str):
+    if status != DAMP_OK:
+        raise DampError(status, where)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensor arguments must be contiguous")
+        return t.data_ptr()
+    if isinstance(t, np.ndarray):
+        if not t.flags["C_CONTIGUOUS"]:
+            raise ValueError("array arguments must be C-contiguous")
+        return t.ctypes.data
+    raise TypeError(f"unsupported argument type {type(t)}")
+
+
+def _cuda(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _stream(stream, device) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+# ---------------------------------------------------------------- host-side calls
+
+def damp_status_string(status: int) -> str:
+    return _lib.damp_status_string(int(status)).decode()
+
+
+def damp_layout(format: int, d_k: int, d_v: int, hp_rows: int) -> tuple[int, int]:
+    """(block_bytes, block_stride) of one (slot, head) block."""
+    b, s = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.damp_layout(format, d_k, d_v, hp_rows, ctypes.byref(b), ctypes.byref(s)),
+           "damp_layout")
+    return b.value, s.value
+
+
+def damp_pool_bytes(format: int, n_slots: int, H: int, d_k: int, d_v: int, hp_rows: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_lib.damp_pool_bytes(format, n_slots, H, d_k, d_v, hp_rows, ctypes.byref(b)),
+           "damp_pool_bytes")
+    return b.value
+
+
+def damp_pool_create(format: int, n_slots: int, H: int, d_k: int, d_v: int, hp_rows: int,
+                     hp_row_idx, dev_buf: torch.Tensor | None) -> int:
+    """Descriptor handle.  hp_row_idx: [H][hp_rows] integer array (host) or None.
+    dev_buf: CUDA uint8 tensor of >= damp_pool_bytes(...) bytes, or None for a
+    host-only descriptor (layout queries and block conversions only)."""
+    idx = None
+    if hp_row_idx is not None and hp_rows > 0:
+        idx = np.ascontiguousarray(np.asarray(hp_row_idx).reshape(H, hp_rows), np.uint16)
+    buf_ptr, nbytes = None, 0
+    if dev_buf is not None:
+        _cuda(dev_buf, torch.uint8, "dev_buf")
+        buf_ptr, nbytes = _ptr(dev_buf), dev_buf.numel()
+    h = ctypes.c_void_p()
+    _check(_lib.damp_pool_create(format, n_slots, H, d_k, d_v, hp_rows, _ptr(idx), buf_ptr,
+                                 nbytes, ctypes.byref(h)), "damp_pool_create")
+    return h.value
+
+
+def damp_pool_destroy(pool: int) -> None:
+    _check(_lib.damp_pool_destroy(pool), "damp_pool_destroy")
+
+
+def damp_pool_block_offset(pool: int, slot: int, h: int) -> int:
+    o = ctypes.c_size_t()
+    _check(_lib.damp_pool_block_offset(pool, slot, h, ctypes.byref(o)), "damp_pool_block_offset")
+    return o.value
+
+
+def damp_block_to_logical(pool: int, h: int, block, fmt: int, d: int) -> dict:
+    """Logical per-row form of one raw block (host bytes)."""
+    block = np.ascontiguousarray(np.frombuffer(bytes(block), np.uint8))
+    if fmt == DAMP_FMT_FP32:
+        f32 = np.empty((d, d), np.float32)
+        _check(_lib.damp_block_to_logical(pool, h, _ptr(block), None, None, None, _ptr(f32)),
+               "damp_block_to_logical")
+        return {"f32": f32}
+    scale = np.empty(d, np.float32)
+    half = np.empty((d, d), np.uint16)
+    code = np.empty((d, d), np.int8)
+    _check(_lib.damp_block_to_logical(pool, h, _ptr(block), _ptr(scale), _ptr(half), _ptr(code),
+                                      None), "damp_block_to_logical")
+    return {"scale": scale, "half": half, "code": code}
+
+
+def damp_block_from_logical(pool: int, h: int, stride: int, scale=None, half=None, code=None,
+                            f32=None) -> np.ndarray:
+    out = np.zeros(stride, np.uint8)
+    c = lambda a, t: None if a is None else np.ascontiguousarray(a, t)
+    scale, half, code, f32 = (c(scale, np.float32), c(half, np.uint16), c(code, np.int8),
+                              c(f32, np.float32))
+    _check(_lib.damp_block_from_logical(pool, h, _ptr(scale), _ptr(half), _ptr(code), _ptr(f32),
+                                        _ptr(out)), "damp_block_from_logical")
+    return out
+
+
+# ---------------------------------------------------------------- device calls
+
+def damp_pool_pack(pool: int, slot_idx: torch.Tensor, state: torch.Tensor, stream=None) -> None:
+    _cuda(slot_idx, torch.int32, "slot_idx")
+    _cuda(state, torch.float32, "state")
+    _check(_lib.damp_pool_pack(pool, slot_idx.numel(), _ptr(slot_idx), _ptr(state),
+                               _stream(stream, state.device)), "damp_pool_pack")
+
+
+def damp_pool_unpack(pool: int, slot_idx: torch.Tensor, state: torch.Tensor, stream=None) -> None:
+    _cuda(slot_idx, torch.int32, "slot_idx")
+    _cuda(state, torch.float32, "state")
+    _check(_lib.damp_pool_unpack(pool, slot_idx.numel(), _ptr(slot_idx), _ptr(state),
+                                 _stream(stream, state.device)), "damp_pool_unpack")
+
+
+def damp_decode_step(pool: int, slot_idx: torch.Tensor, q: torch.Tensor, k: torch.Tensor,
+                     v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
+                     stream=None) -> None:
+    """One decode step.  q, k [n][H][d_k] and v [n][H][d_v] in bf16 or fp32;
+    alpha fp32 [n][H] (GDN) or [n][H][d_k] (KDA); beta fp32 [n][H]; out fp32
+    [n][H][d_v]."""
+    _cuda(slot_idx, torch.int32, "slot_idx")
+    _cuda(q, None, "q")
+    if q.dtype == torch.bfloat16:
+        dt = DAMP_DTYPE_BF16
+    elif q.dtype == torch.float32:
+        dt = DAMP_DTYPE_F32
+    else:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    _cuda(k, q.dtype, "k")
+    _cuda(v, q.dtype, "v")
+    _cuda(alpha, torch.float32, "alpha")
+    _cuda(beta, torch.float32, "beta")
+    _cuda(out, torch.float32, "out")
+    gate = DAMP_GATE_VECTOR if alpha.dim() == 3 else DAMP_GATE_SCALAR
+    _check(_lib.damp_decode_step(pool, slot_idx.numel(), _ptr(slot_idx), dt, _ptr(q), _ptr(k),
+                                 _ptr(v), gate, _ptr(alpha), _ptr(beta), _ptr(out),
+                                 _stream(stream, q.device)), "damp_decode_step")
+
+
+def damp_pool_get_error(pool: int, clear: bool = False, stream=None, device=None) -> int:
+    f = ctypes.c_uint32()
+    _check(_lib.damp_pool_get_error(pool, ctypes.byref(f), int(bool(clear)),
+                                    _stream(stream, device)), "damp_pool_get_error")
+    return f.value
+
+
+# ---------------------------------------------------------------- convenience
+
+class DampPool:
+    """A pool buffer (allocated by PyTorch) bound to a libdamp descriptor."""
+
+    def __init__(self, fmt, n_slots: int, H: int, d: int, hp_row_idx=None,
+                 device="cuda"):
+        self.fmt = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+        hp_row_idx = None if hp_row_idx is None else np.asarray(hp_row_idx).reshape(H, -1)
+        self.hp = 0 if hp_row_idx is None else hp_row_idx.shape[1]
+        self.n_slots, self.H, self.d = n_slots, H, d
+        self.block_bytes, self.block_stride = damp_layout(self.fmt, d, d, self.hp)
+        self.nbytes = damp_pool_bytes(self.fmt, n_slots, H, d, d, self.hp)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        self.handle = damp_pool_create(self.fmt, n_slots, H, d, d, self.hp, hp_row_idx, self.buf)
+        self.header_bytes = damp_pool_block_offset(self.handle, 0, 0)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            damp_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def blocks(self) -> torch.Tensor:
+        """View of the block area: uint8 [n_slots][H][block_stride]."""
+        return self.buf[self.header_bytes:].view(self.n_slots, self.H, self.block_stride)
+
+    def pack(self, slot_idx, state, stream=None):
+        damp_pool_pack(self.handle, slot_idx, state, stream)
+
+    def unpack(self, slot_idx, state, stream=None):
+        damp_pool_unpack(self.handle, slot_idx, state, stream)
+
+    def step(self, slot_idx, q, k, v, alpha, beta, out, stream=None):
+        damp_decode_step(self.handle, slot_idx, q, k, v, alpha, beta, out, stream)
+
+    def get_error(self, clear=False, stream=None) -> int:
+        return damp_pool_get_error(self.handle, clear, stream, self.buf.device)
+
+    def read_logical(self, slots=None) -> dict:
+        """Logical form of blocks [len(slots)][H] (host numpy), via one D2H copy."""
+        raw = self.blocks().cpu().numpy()
+        slots = range(self.n_slots) if slots is None else slots
+        out = None
+        for i, s in enumerate(slots):
+            for h in range(self.H):
+                lg = damp_block_to_logical(self.handle, h, raw[s, h], self.fmt, self.d)
+                if out is None:
+                    out = {k: np.empty((len(slots), self.H) + v.shape, v.dtype)
+                           for k, v in lg.items()}
+                for k_, v_ in lg.items():
+                    out[k_][i, h] = v_
+        return out
+
+    def write_logical(self, slot: int, logical: dict):
+        """Write the logical form [H][...] of one slot into the pool (host -> device)."""
+        raw = np.stack([damp_block_from_logical(self.handle, h, self.block_stride,
+                                                **{k: v[h] for k, v in logical.items()})
+                        for h in range(self.H)])
+        self.blocks()[slot].copy_(torch.from_numpy(raw))

@@ -1,0 +1,327 @@
+// damp_abi.cu -- the C ABI of libdamp (declared in include/damp.h).
+//
+// Host-side argument checks, the pool descriptor and its header, the block
+// layout, and the host-only conversions between raw blocks and the logical
+// per-row form.  Every check happens before anything is enqueued; kernels
+// report device-side conditions through the pool's status word.
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "../../include/damp.h"
+#include "damp_internal.h"
+
+using damp::PoolDesc;
+
+struct damp_pool {
+    PoolDesc d;
+};
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int format, int d_k, int d_v, int hp_rows) {
+    if (format != DAMP_FMT_FP32 && format != DAMP_FMT_INT8_ROW && format != DAMP_FMT_MIXED)
+        return DAMP_ERR_INVALID_ARGUMENT;
+    if (hp_rows < 0 || hp_rows > d_k) return DAMP_ERR_INVALID_ARGUMENT;
+    if (format != DAMP_FMT_MIXED && hp_rows != 0) return DAMP_ERR_INVALID_ARGUMENT;
+    if (d_k != d_v) return DAMP_ERR_UNSUPPORTED;
+    if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return DAMP_ERR_UNSUPPORTED;
+    return DAMP_OK;
+}
+
+void layout(int format, int d, int hp, size_t* bytes, size_t* stride, uint32_t* f16_off,
+            uint32_t* i8_off) {
+    if (format == DAMP_FMT_FP32) {
+        *bytes = (size_t)d * d * 4;
+        *stride = *bytes;
+        *f16_off = *i8_off = 0;
+        return;
+    }
+    const size_t r = (size_t)(d - hp);
+    *bytes = 4 * r + 2 * (size_t)hp * d + r * d;
+    const size_t scales = align_up(4 * r, 16);
+    *f16_off = (uint32_t)scales;
+    *i8_off = (uint32_t)(scales + 2 * (size_t)hp * d);
+    *stride = align_up(scales + 2 * (size_t)hp * d + r * d, 16);
+}
+
+size_t header_bytes(int H) {
+    return align_up(damp::kStatusBytes + (size_t)H * damp::kMaskWords * 4, 256);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? DAMP_OK : DAMP_ERR_CUDA; }
+
+bool is_fp16_row(const PoolDesc& d, int h, int i) {
+    return (d.host_masks[(size_t)h * damp::kMaskWords + (i >> 5)] >> (i & 31)) & 1u;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* damp_status_string(int status) {
+    switch (status) {
+        case DAMP_OK: return "ok";
+        case DAMP_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case DAMP_ERR_UNSUPPORTED: return "unsupported shape (d_k == d_v in {16, 32, 64, 128})";
+        case DAMP_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case DAMP_ERR_BUFFER_TOO_SMALL: return "pool buffer too small";
+        case DAMP_ERR_CUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
+                size_t* block_stride) {
+    const int rc = check_shape(format, d_k, d_v, hp_rows);
+    if (rc) return rc;
+    size_t b, s;
+    uint32_t f, i;
+    layout(format, d_k, hp_rows, &b, &s, &f, &i);
+    if (block_bytes) *block_bytes = b;
+    if (block_stride) *block_stride = s;
+    return DAMP_OK;
+}
+
+int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
+                    size_t* bytes) {
+    if (!bytes || n_slots < 1 || H < 1) return DAMP_ERR_INVALID_ARGUMENT;
+    const int rc = check_shape(format, d_k, d_v, hp_rows);
+    if (rc) return rc;
+    size_t b, s;
+    uint32_t f, i;
+    layout(format, d_k, hp_rows, &b, &s, &f, &i);
+    *bytes = header_bytes(H) + (size_t)n_slots * H * s;
+    return DAMP_OK;
+}
+
+int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
+                     const uint16_t* hp_row_idx, void* dev_buf, size_t buf_bytes,
+                     damp_pool** out) {
+    if (!out) return DAMP_ERR_INVALID_ARGUMENT;
+    *out = nullptr;
+    if (n_slots < 1 || H < 1) return DAMP_ERR_INVALID_ARGUMENT;
+    int rc = check_shape(format, d_k, d_v, hp_rows);
+    if (rc) return rc;
+    if (hp_rows > 0 && !hp_row_idx) return DAMP_ERR_INVALID_ARGUMENT;
+    std::vector<uint32_t> masks((size_t)H * damp::kMaskWords, 0u);
+    for (int h = 0; h < H; ++h)
+        for (int j = 0; j < hp_rows; ++j) {
+            const int i = hp_row_idx[(size_t)h * hp_rows + j];
+            if (i >= d_k) return DAMP_ERR_INVALID_ARGUMENT;
+            uint32_t& w = masks[(size_t)h * damp::kMaskWords + (i >> 5)];
+            if (w & (1u << (i & 31))) return DAMP_ERR_INVALID_ARGUMENT;  // repeated row
+            w |= 1u << (i & 31);
+        }
+    PoolDesc d{};
+    d.format = format;
+    d.n_slots = n_slots;
+    d.H = H;
+    d.d = d_k;
+    d.hp = hp_rows;
+    layout(format, d_k, hp_rows, &d.block_bytes, &d.block_stride, &d.f16_off, &d.i8_off);
+    d.header_bytes = header_bytes(H);
+    d.pool_bytes = d.header_bytes + (size_t)n_slots * H * d.block_stride;
+    if (dev_buf) {
+        if (!aligned16(dev_buf)) return DAMP_ERR_MISALIGNED;
+        if (buf_bytes < d.pool_bytes) return DAMP_ERR_BUFFER_TOO_SMALL;
+    }
+    damp_pool* p = new (std::nothrow) damp_pool;
+    if (!p) return DAMP_ERR_INVALID_ARGUMENT;
+    p->d = d;
+    p->d.dev_buf = static_cast<uint8_t*>(dev_buf);
+    p->d.host_masks = new (std::nothrow) uint32_t[masks.size()];
+    if (!p->d.host_masks) {
+        delete p;
+        return DAMP_ERR_INVALID_ARGUMENT;
+    }
+    memcpy(p->d.host_masks, masks.data(), masks.size() * 4);
+    if (dev_buf) {
+        std::vector<uint8_t> hdr(d.header_bytes, 0);
+        memcpy(hdr.data() + damp::kStatusBytes, masks.data(), masks.size() * 4);
+        const cudaError_t e = cudaMemcpy(dev_buf, hdr.data(), hdr.size(), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            delete[] p->d.host_masks;
+            delete p;
+            return DAMP_ERR_CUDA;
+        }
+    }
+    *out = p;
+    return DAMP_OK;
+}
+
+int damp_pool_destroy(damp_pool* pool) {
+    if (!pool) return DAMP_OK;
+    delete[] pool->d.host_masks;
+    delete pool;
+    return DAMP_OK;
+}
+
+int damp_pool_block_offset(const damp_pool* pool, int slot, int h, size_t* offset) {
+    if (!pool || !offset) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    if (slot < 0 || slot >= d.n_slots || h < 0 || h >= d.H) return DAMP_ERR_INVALID_ARGUMENT;
+    *offset = d.header_bytes + ((size_t)slot * d.H + h) * d.block_stride;
+    return DAMP_OK;
+}
+
+static int codec_args(const damp_pool* pool, int n, const int32_t* slot_idx, const float* state,
+                      damp::CodecArgs* a) {
+    if (!pool || n < 0) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    if (!d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
+    if (n == 0) return 1;  // nothing to do
+    if (!slot_idx || !state) return DAMP_ERR_INVALID_ARGUMENT;
+    if (!aligned16(state) || (reinterpret_cast<uintptr_t>(slot_idx) & 3u))
+        return DAMP_ERR_MISALIGNED;
+    a->blocks = d.dev_buf + d.header_bytes;
+    a->masks = reinterpret_cast<const uint32_t*>(d.dev_buf + damp::kStatusBytes);
+    a->status = reinterpret_cast<uint32_t*>(d.dev_buf);
+    a->slot_idx = slot_idx;
+    a->state = const_cast<float*>(state);
+    a->n = n;
+    a->H = d.H;
+    a->n_slots = d.n_slots;
+    a->hp = d.hp;
+    a->block_stride = (uint32_t)d.block_stride;
+    a->f16_off = d.f16_off;
+    a->i8_off = d.i8_off;
+    const int upi = 128 / d.d;
+    a->n_items = (int)(((size_t)n * d.H + upi - 1) / upi);
+    return DAMP_OK;
+}
+
+int damp_pool_pack(const damp_pool* pool, int n, const int32_t* slot_idx, const float* state,
+                   void* stream) {
+    damp::CodecArgs a{};
+    const int rc = codec_args(pool, n, slot_idx, state, &a);
+    if (rc) return rc < 0 ? rc : DAMP_OK;
+    return cuda_status(damp::launch_pack(pool->d, a, static_cast<cudaStream_t>(stream)));
+}
+
+int damp_pool_unpack(const damp_pool* pool, int n, const int32_t* slot_idx, float* state,
+                     void* stream) {
+    damp::CodecArgs a{};
+    const int rc = codec_args(pool, n, slot_idx, state, &a);
+    if (rc) return rc < 0 ? rc : DAMP_OK;
+    return cuda_status(damp::launch_unpack(pool->d, a, static_cast<cudaStream_t>(stream)));
+}
+
+int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int in_dtype,
+                     const void* q, const void* k, const void* v, int gate, const float* alpha,
+                     const float* beta, float* out, void* stream) {
+    if (!pool || n < 0) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    if (!d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
+    if (in_dtype != DAMP_DTYPE_BF16 && in_dtype != DAMP_DTYPE_F32) return DAMP_ERR_INVALID_ARGUMENT;
+    if (gate != DAMP_GATE_SCALAR && gate != DAMP_GATE_VECTOR) return DAMP_ERR_INVALID_ARGUMENT;
+    if (n == 0) return DAMP_OK;
+    if (!slot_idx || !q || !k || !v || !alpha || !beta || !out) return DAMP_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return DAMP_ERR_MISALIGNED;
+    if (gate == DAMP_GATE_VECTOR && !aligned16(alpha)) return DAMP_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(slot_idx) & 3u) || (reinterpret_cast<uintptr_t>(beta) & 3u) ||
+        (reinterpret_cast<uintptr_t>(alpha) & 3u))
+        return DAMP_ERR_MISALIGNED;
+    if ((size_t)n * d.H > (size_t)0x7fffffff) return DAMP_ERR_UNSUPPORTED;
+    damp::StepArgs a{};
+    a.blocks = d.dev_buf + d.header_bytes;
+    a.masks = reinterpret_cast<const uint32_t*>(d.dev_buf + damp::kStatusBytes);
+    a.status = reinterpret_cast<uint32_t*>(d.dev_buf);
+    a.slot_idx = slot_idx;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.out = out;
+    a.n = n;
+    a.H = d.H;
+    a.n_slots = d.n_slots;
+    a.hp = d.hp;
+    a.block_stride = (uint32_t)d.block_stride;
+    a.f16_off = d.f16_off;
+    a.i8_off = d.i8_off;
+    const int upi = 128 / d.d;
+    a.n_items = (int)(((size_t)n * d.H + upi - 1) / upi);
+    return cuda_status(
+        damp::launch_decode_step(d, a, in_dtype, gate, static_cast<cudaStream_t>(stream)));
+}
+
+int damp_pool_get_error(const damp_pool* pool, uint32_t* flags, int clear, void* stream) {
+    if (!pool || !flags || !pool->d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* st = reinterpret_cast<uint32_t*>(pool->d.dev_buf);
+    uint32_t host = 0;
+    cudaError_t e = cudaMemcpyAsync(&host, st, 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(st, 0, 4, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return DAMP_ERR_CUDA;
+    *flags = host;
+    return DAMP_OK;
+}
+
+int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float* scale,
+                          uint16_t* half, int8_t* code, float* f32) {
+    if (!pool || !block || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    const uint8_t* b = static_cast<const uint8_t*>(block);
+    const int D = d.d;
+    if (d.format == DAMP_FMT_FP32) {
+        if (!f32) return DAMP_ERR_INVALID_ARGUMENT;
+        memcpy(f32, b, (size_t)D * D * 4);
+        return DAMP_OK;
+    }
+    if (!scale || !half || !code) return DAMP_ERR_INVALID_ARGUMENT;
+    int r16 = 0, r8 = 0;
+    for (int i = 0; i < D; ++i) {
+        if (is_fp16_row(d, h, i)) {
+            scale[i] = 0.0f;
+            memcpy(half + (size_t)i * D, b + d.f16_off + (size_t)r16 * 2 * D, (size_t)2 * D);
+            memset(code + (size_t)i * D, 0, D);
+            ++r16;
+        } else {
+            memcpy(&scale[i], b + (size_t)r8 * 4, 4);
+            memcpy(code + (size_t)i * D, b + d.i8_off + (size_t)r8 * D, D);
+            memset(half + (size_t)i * D, 0, (size_t)2 * D);
+            ++r8;
+        }
+    }
+    return DAMP_OK;
+}
+
+int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
+                            const uint16_t* half, const int8_t* code, const float* f32,
+                            void* block) {
+    if (!pool || !block || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    uint8_t* b = static_cast<uint8_t*>(block);
+    const int D = d.d;
+    if (d.format == DAMP_FMT_FP32) {
+        if (!f32) return DAMP_ERR_INVALID_ARGUMENT;
+        memcpy(b, f32, (size_t)D * D * 4);
+        return DAMP_OK;
+    }
+    if (!scale || !half || !code) return DAMP_ERR_INVALID_ARGUMENT;
+    memset(b, 0, d.block_stride);
+    int r16 = 0, r8 = 0;
+    for (int i = 0; i < D; ++i) {
+        if (is_fp16_row(d, h, i)) {
+            memcpy(b + d.f16_off + (size_t)r16 * 2 * D, half + (size_t)i * D, (size_t)2 * D);
+            ++r16;
+        } else {
+            memcpy(b + (size_t)r8 * 4, &scale[i], 4);
+            memcpy(b + d.i8_off + (size_t)r8 * D, code + (size_t)i * D, D);
+            ++r8;
+        }
+    }
+    return DAMP_OK;
+}
+
+}  // extern "C"

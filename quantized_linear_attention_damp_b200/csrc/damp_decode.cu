@@ -1,0 +1,447 @@
+// damp_decode.cu -- the decode-step kernel of libdamp (sm_100a).
+//
+// One decode step of a DAMP-style compressed recurrent state for every
+// (batch entry, head) unit ("DAMP: Decay-Aware Mixed-Precision Recurrent-State
+// Quantization", both abstracts; step order of "STEPQuant ...", Appendix
+// Table C2, steps 1, 2, 3 and 6):
+//   reconstruct S^ (FP16 rows exact, INT8 rows code*scale)      step 1
+//   S' = D S^, u = k^T S', X = S' + (beta k)(v - u)^T           step 2
+//   out = X^T q, before requantization                          step 3
+//   requantize X in place (FP16 rows, INT8 rows + FP32 scale)   step 6
+//
+// Work decomposition.  A persistent CTA of 9 warps walks work items (128/d
+// units each) with a grid stride.  Warp 8 is the producer: it reads the
+// per-unit metadata (slot, gates), waits until a shared-memory stage is free
+// and moves the unit's state block and inputs into it with cp.async.bulk
+// (no tensor map, no multicast), completing on the stage's "full" mbarrier.
+// Warps 0-7 consume: each thread keeps a (d/8) x 4 tile of the state in
+// registers from the dequantize through the requantize, so shared memory is
+// read once and written once per unit.  The new block is written back into
+// the same stage and thread 0 streams it to HBM with one bulk store, then
+// frees the stage one item later (after the store has read shared memory).
+// The in-place update is safe because a unit's block has exactly one reader
+// and one writer per call (Table C2 step 6: the old representation stays
+// valid until its reader is done) -- slot indices within a call are distinct.
+//
+// Numerics.  u_j is summed in the recursive pairwise order over key rows:
+// each thread sums its d/8 consecutive rows as a subtree, the 8 row-group
+// sums are combined by the top three levels of the same tree.  Together with
+// the explicit round-to-nearest intrinsics (and -fmad=false) this makes X,
+// and so every stored code, FP16 value and scale, a deterministic function of
+// the inputs.  The readout uses out_j = w_j + c*delta_j with
+// w = S'^T q and c = q^T (beta k), which equals X^T q up to FP32 rounding.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/damp.h"
+#include "damp_device.cuh"
+
+namespace damp {
+namespace {
+
+constexpr int kConsumerThreads = 256;
+constexpr int kThreads = 288;
+
+struct Meta {  // one per unit in a stage, written by the producer
+    int slot;
+    float alpha;  // GDN scalar decay
+    float beta;
+    int exists;   // unit index < n*H
+};
+
+template <bool BF16>
+__device__ __forceinline__ float load_in(const uint8_t* base, int idx) {
+    if constexpr (BF16) {
+        const uint16_t h = reinterpret_cast<const uint16_t*>(base)[idx];
+        return __uint_as_float(static_cast<uint32_t>(h) << 16);
+    } else {
+        return reinterpret_cast<const float*>(base)[idx];
+    }
+}
+
+template <int D, bool QUANT, bool KDA, bool BF16>
+__global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
+    using G = Geo<D>;
+    constexpr int RPT = G::RPT, UPI = G::UPI, LPR = G::LPR;
+    constexpr int LOGR = (RPT == 2) ? 1 : (RPT == 4) ? 2 : (RPT == 8) ? 3 : 4;
+    constexpr uint32_t ELT = BF16 ? 2 : 4;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int NS = a.n_stages;
+    const uint32_t bar0 = smem_u32(smem + a.bar_off);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int n_units = a.n * a.H;
+
+    // ------------------------------------------------------------------ producer
+    if (warp == 8) {
+        auto load_meta = [&](int item) {
+            Meta m{-1, 0.f, 0.f, 0};
+            const int u = item * UPI + lane;
+            if (lane < UPI && item < a.n_items && u < n_units) {
+                m.exists = 1;
+                m.slot = __ldg(a.slot_idx + u / a.H);
+                if constexpr (!KDA) m.alpha = __ldg(a.alpha + u);
+                m.beta = __ldg(a.beta + u);
+            }
+            return m;
+        };
+        int it = 0;
+        Meta cur = load_meta(blockIdx.x);
+        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x, ++it) {
+            const Meta nxt = load_meta(item + gridDim.x);  // prefetch one item ahead
+            const int stage = it % NS;
+            const uint32_t fill = static_cast<uint32_t>(it / NS);
+            bool ok = true;
+            if (fill > 0) ok = mbar_wait_bounded(empty_bar(stage), (fill - 1) & 1u);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
+                break;
+            }
+            uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+            const int u = item * UPI + lane;
+            const bool load = cur.exists && cur.slot >= 0 && cur.slot < a.n_slots;
+            uint32_t tx = 0;
+            if (lane < UPI) {
+                *reinterpret_cast<Meta*>(st + a.st_meta + lane * sizeof(Meta)) = cur;
+                if (load) tx = a.block_stride + 3u * D * ELT + (KDA ? 4u * D : 0u) + 16u;
+            }
+            const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
+            __syncwarp();
+            if (lane == 0) {
+                if (tx_all) mbar_arrive_expect_tx(full_bar(stage), tx_all);
+                else mbar_arrive(full_bar(stage));
+            }
+            __syncwarp();
+            if (load) {
+                const int h = u % a.H;
+                const uint32_t fb = full_bar(stage);
+                const uint8_t* gblk =
+                    a.blocks + ((size_t)cur.slot * a.H + h) * (size_t)a.block_stride;
+                bulk_g2s(smem_u32(st + lane * a.block_stride), gblk, a.block_stride, fb);
+                const size_t io = (size_t)u * D * ELT;
+                bulk_g2s(smem_u32(st + a.st_q + lane * D * ELT),
+                         static_cast<const uint8_t*>(a.q) + io, D * ELT, fb);
+                bulk_g2s(smem_u32(st + a.st_k + lane * D * ELT),
+                         static_cast<const uint8_t*>(a.k) + io, D * ELT, fb);
+                bulk_g2s(smem_u32(st + a.st_v + lane * D * ELT),
+                         static_cast<const uint8_t*>(a.v) + io, D * ELT, fb);
+                if constexpr (KDA)
+                    bulk_g2s(smem_u32(st + a.st_alpha + lane * D * 4), a.alpha + (size_t)u * D,
+                             D * 4, fb);
+                bulk_g2s(smem_u32(st + a.st_mask + lane * 16), a.masks + (size_t)h * kMaskWords,
+                         16, fb);
+            }
+            cur = nxt;
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------------ consumers
+    const int ui = tid / G::TPU;        // unit within the item
+    const int tu = tid % G::TPU;        // thread within the unit
+    const int cg = tu % LPR;            // column group: columns 4cg..4cg+3
+    const int rg = tu / LPR;            // row group: rows r0..r0+RPT-1
+    const int r0 = rg * RPT;
+
+    uint8_t* scratch = smem + a.scratch_off;
+    float* red_u = reinterpret_cast<float*>(scratch);                  // [UPI][8][D]
+    float* red_w = red_u + UPI * 8 * D;                                // [UPI][8][D]
+    float* delta_s = red_w + UPI * 8 * D;                              // [UPI][D]
+    float* cpart_s = delta_s + UPI * D;                                // [UPI][8]
+    float* rowbuf = cpart_s + UPI * 8 + (ui * 8 + rg) * 2 * RPT;       // this row group's
+
+    int it = 0;
+    bool aborted = false;
+    for (int item = blockIdx.x; item < a.n_items; item += gridDim.x, ++it) {
+        const int stage = it % NS;
+        const uint32_t parity = static_cast<uint32_t>(it / NS) & 1u;
+        const bool ok = mbar_wait_bounded(full_bar(stage), parity);
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const Meta meta = *reinterpret_cast<const Meta*>(st + a.st_meta + ui * sizeof(Meta));
+        const int u = item * UPI + ui;
+        const bool active = ok && meta.exists && meta.slot >= 0 && meta.slot < a.n_slots;
+        uint8_t* blk = st + ui * a.block_stride;
+        const uint8_t* sq = st + a.st_q + ui * D * ELT;
+        const uint8_t* sk = st + a.st_k + ui * D * ELT;
+        const float* salpha = reinterpret_cast<const float*>(st + a.st_alpha) + ui * D;
+
+        float2 x[RPT][2];
+        uint32_t bits = 0;
+        int rank16 = 0;
+        if (active) {
+            // ---- step 1: reconstruct, then D_t S^
+            if constexpr (QUANT) {
+                const uint4 mw = *reinterpret_cast<const uint4*>(st + a.st_mask + ui * 16);
+                row_formats<D>(mw, r0, bits, rank16);
+                load_quant_tile<D>(blk, a.f16_off, a.i8_off, bits, rank16, r0, cg, x);
+            } else {
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    const float4 f = *reinterpret_cast<const float4*>(
+                        blk + ((size_t)(r0 + i) * D + 4 * cg) * 4);
+                    x[i][0] = make_float2(f.x, f.y);
+                    x[i][1] = make_float2(f.z, f.w);
+                }
+            }
+            // ---- step 2 (first half): u = k^T S' (pairwise), w = q^T S', c = q^T (beta k)
+            float2 stk[LOGR][2];
+            float2 usum0 = f2(0.f), usum1 = f2(0.f);
+            float2 w0 = f2(0.f), w1 = f2(0.f);
+            float cp = 0.f;
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = r0 + i;
+                const float al = KDA ? salpha[r] : meta.alpha;
+                x[i][0] = __fmul2_rn(x[i][0], f2(al));
+                x[i][1] = __fmul2_rn(x[i][1], f2(al));
+                const float kr = load_in<BF16>(sk, r);
+                const float qr = load_in<BF16>(sq, r);
+                float2 v0 = __fmul2_rn(f2(kr), x[i][0]);
+                float2 v1 = __fmul2_rn(f2(kr), x[i][1]);
+#pragma unroll
+                for (int b = 0; b < LOGR; ++b) {
+                    if ((i >> b) & 1) {
+                        v0 = __fadd2_rn(stk[b][0], v0);
+                        v1 = __fadd2_rn(stk[b][1], v1);
+                    } else {
+                        stk[b][0] = v0;
+                        stk[b][1] = v1;
+                        break;
+                    }
+                }
+                if (i == RPT - 1) {
+                    usum0 = v0;
+                    usum1 = v1;
+                }
+                w0 = __ffma2_rn(f2(qr), x[i][0], w0);
+                w1 = __ffma2_rn(f2(qr), x[i][1], w1);
+                cp = __fmaf_rn(qr, __fmul_rn(meta.beta, kr), cp);
+            }
+            float* ru = red_u + (ui * 8 + rg) * D + 4 * cg;
+            float* rw = red_w + (ui * 8 + rg) * D + 4 * cg;
+            *reinterpret_cast<float4*>(ru) = make_float4(usum0.x, usum0.y, usum1.x, usum1.y);
+            *reinterpret_cast<float4*>(rw) = make_float4(w0.x, w0.y, w1.x, w1.y);
+            if (cg == 0) cpart_s[ui * 8 + rg] = cp;
+        }
+        if (bar_red_or(1, kConsumerThreads, ok ? 0 : 1)) {
+            aborted = true;
+            break;
+        }
+
+        // ---- step 2 (second half) + step 3: per column j, delta_j and out_j
+        if (tu < D) {
+            const int j = tu;
+            if (active) {
+                const float* cu = red_u + ui * 8 * D + j;
+                const float* cw = red_w + ui * 8 * D + j;
+                const float uj = __fadd_rn(__fadd_rn(__fadd_rn(cu[0 * D], cu[1 * D]),
+                                                     __fadd_rn(cu[2 * D], cu[3 * D])),
+                                           __fadd_rn(__fadd_rn(cu[4 * D], cu[5 * D]),
+                                                     __fadd_rn(cu[6 * D], cu[7 * D])));
+                float wj = 0.f, c = 0.f;
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    wj = __fadd_rn(wj, cw[g * D]);
+                    c = __fadd_rn(c, cpart_s[ui * 8 + g]);
+                }
+                const float vj = load_in<BF16>(st + a.st_v + ui * D * ELT, j);
+                const float dj = __fsub_rn(vj, uj);
+                delta_s[ui * D + j] = dj;
+                a.out[(size_t)u * D + j] = __fmaf_rn(c, dj, wj);
+            } else if (meta.exists) {
+                a.out[(size_t)u * D + j] = 0.f;
+                if (j == 0 && meta.slot >= a.n_slots) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
+            }
+        }
+        bar_sync(1, kConsumerThreads);
+
+        // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
+        if (active) {
+            const float4 dl = *reinterpret_cast<const float4*>(delta_s + ui * D + 4 * cg);
+            const float2 d0 = make_float2(dl.x, dl.y), d1 = make_float2(dl.z, dl.w);
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const float b = __fmul_rn(meta.beta, load_in<BF16>(sk, r0 + i));
+                x[i][0] = __ffma2_rn(f2(b), d0, x[i][0]);
+                x[i][1] = __ffma2_rn(f2(b), d1, x[i][1]);
+            }
+            if constexpr (QUANT) {
+                store_quant_tile<D>(blk, a.f16_off, a.i8_off, bits, rank16, r0, cg, x, rowbuf);
+            } else {
+#pragma unroll
+                for (int i = 0; i < RPT; ++i)
+                    *reinterpret_cast<float4*>(blk + ((size_t)(r0 + i) * D + 4 * cg) * 4) =
+                        make_float4(x[i][0].x, x[i][0].y, x[i][1].x, x[i][1].y);
+            }
+            fence_proxy_async_smem();
+        }
+        bar_sync(1, kConsumerThreads);
+
+        // ---- write back and recycle the previous stage
+        if (tid == 0) {
+#pragma unroll
+            for (int w = 0; w < UPI; ++w) {
+                const Meta m = *reinterpret_cast<const Meta*>(st + a.st_meta + w * sizeof(Meta));
+                if (m.exists && m.slot >= 0 && m.slot < a.n_slots) {
+                    const int uw = item * UPI + w;
+                    uint8_t* gblk = a.blocks + ((size_t)m.slot * a.H + uw % a.H) *
+                                                   (size_t)a.block_stride;
+                    bulk_s2g(gblk, smem_u32(st + w * a.block_stride), a.block_stride);
+                }
+            }
+            bulk_commit();
+            if (it > 0) {
+                bulk_wait_read<1>();
+                mbar_arrive(empty_bar((it - 1) % NS));
+            }
+        }
+    }
+
+    if (tid == 0) {
+        if (aborted) {
+            atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
+            // drain copies that may still be landing in this CTA's stages
+            for (int j = 0; j < NS; ++j) {
+                const int jt = it + j;
+                const int item = blockIdx.x + jt * gridDim.x;
+                if (item >= a.n_items) break;
+                (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
+                                        100000000ull);
+            }
+        }
+        bulk_wait_all<0>();
+    }
+}
+
+// ---------------------------------------------------------------------- host
+
+struct Layout {
+    uint32_t stage_bytes, st_q, st_k, st_v, st_alpha, st_mask, st_meta;
+    uint32_t scratch_bytes;
+};
+
+inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+Layout stage_layout(int d, uint32_t stride, int in_dtype, int gate) {
+    const uint32_t upi = 128 / d, elt = (in_dtype == DAMP_DTYPE_BF16) ? 2 : 4;
+    Layout L{};
+    uint32_t off = upi * stride;
+    L.st_q = off;
+    off = align_up(off + upi * d * elt, 16);
+    L.st_k = off;
+    off = align_up(off + upi * d * elt, 16);
+    L.st_v = off;
+    off = align_up(off + upi * d * elt, 16);
+    L.st_alpha = off;
+    off += (gate == DAMP_GATE_VECTOR) ? upi * d * 4 : 0;
+    L.st_mask = off;
+    off += upi * 16;
+    L.st_meta = off;
+    off += upi * sizeof(Meta);
+    L.stage_bytes = align_up(off, 128);
+    // red_u + red_w [128/d][8][d] each, delta [128], cpart [8*128/d], rowbuf 2*128
+    L.scratch_bytes = align_up((2 * 8 * 128 + 128 + 8 * upi + 2 * 128) * 4, 128);
+    return L;
+}
+
+template <int D, bool QUANT, bool KDA, bool BF16>
+cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    auto kern = decode_step_kernel<D, QUANT, KDA, BF16>;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        227 * 1024);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            100);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+
+    StepArgs a = a0;
+    int dev = 0, sms = 0, smem_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                    dev)) != cudaSuccess)
+        return e;
+    const Layout L = stage_layout(D, a.block_stride, BF16 ? DAMP_DTYPE_BF16 : DAMP_DTYPE_F32,
+                                  KDA ? DAMP_GATE_VECTOR : DAMP_GATE_SCALAR);
+    // Two CTAs per SM when at least three stages fit, else one CTA with as many
+    // stages as fit (up to 8).
+    const uint32_t per_cta_2 = static_cast<uint32_t>(smem_sm) / 2 - 1024;
+    const uint32_t per_cta_1 = 227u * 1024u;
+    auto stages_for = [&](uint32_t budget) {
+        const uint32_t fixed = L.scratch_bytes + 128;
+        if (budget <= fixed) return 0u;
+        uint32_t ns = (budget - fixed) / L.stage_bytes;
+        return ns > 8 ? 8u : ns;
+    };
+    uint32_t ns = stages_for(per_cta_2);
+    if (ns < 3) ns = stages_for(per_cta_1);
+    if (ns < 2) return cudaErrorInvalidConfiguration;
+    a.n_stages = static_cast<int>(ns);
+    a.stage_bytes = L.stage_bytes;
+    a.st_q = L.st_q;
+    a.st_k = L.st_k;
+    a.st_v = L.st_v;
+    a.st_alpha = L.st_alpha;
+    a.st_mask = L.st_mask;
+    a.st_meta = L.st_meta;
+    a.scratch_off = ns * L.stage_bytes;
+    a.bar_off = a.scratch_off + L.scratch_bytes;
+    const size_t smem = a.bar_off + 16u * ns;
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) !=
+        cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int grid = std::min(a.n_items, sms * per_sm);
+    kern<<<grid, kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_fmt(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
+                         cudaStream_t s) {
+    const bool q = p.format != DAMP_FMT_FP32, kda = gate == DAMP_GATE_VECTOR,
+               bf = in_dtype == DAMP_DTYPE_BF16;
+    if (q) {
+        if (kda) return bf ? launch_t<D, true, true, true>(a, s) : launch_t<D, true, true, false>(a, s);
+        return bf ? launch_t<D, true, false, true>(a, s) : launch_t<D, true, false, false>(a, s);
+    }
+    if (kda) return bf ? launch_t<D, false, true, true>(a, s) : launch_t<D, false, true, false>(a, s);
+    return bf ? launch_t<D, false, false, true>(a, s) : launch_t<D, false, false, false>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
+                               cudaStream_t stream) {
+    switch (p.d) {
+        case 16: return dispatch_fmt<16>(p, a, in_dtype, gate, stream);
+        case 32: return dispatch_fmt<32>(p, a, in_dtype, gate, stream);
+        case 64: return dispatch_fmt<64>(p, a, in_dtype, gate, stream);
+        case 128: return dispatch_fmt<128>(p, a, in_dtype, gate, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace damp

@@ -1,0 +1,290 @@
+// damp_device.cuh -- device helpers of libdamp: PTX wrappers for the bulk-copy
+// pipeline and the per-thread tile codec (dequantize / requantize) shared by
+// the decode-step and pack/unpack kernels.
+//
+// Arithmetic contract (every FP32 operation is written with an explicit
+// round-to-nearest intrinsic and the library is built with -fmad=false, so no
+// multiply-add is contracted behind our back):
+//   FP16 row   : S^ = (float)h                         exact
+//   INT8 row   : S^ = fl(code * scale)                 one rounding
+//   requantize : FP16  h = RN16(x)  (cvt.rn, IEEE overflow to inf)
+//                INT8  a = max|x| over the row; scale = fl(a/127);
+//                      inv = fl(127/a); code = RNE(x*inv) taken from ONE fused
+//                      multiply-add with 1.5*2^23 (exact RNE of the exact
+//                      product, see quantize4); a == 0 or inv == inf -> 0.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "damp_internal.h"
+
+namespace damp {
+
+// ----------------------------------------------------------------------------
+// PTX wrappers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t tx) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(tx)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Every wait in the pipeline is bounded: after kWaitNs it gives up and the
+// caller records DAMP_EFLAG_TIMEOUT instead of spinning forever.
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+// global -> shared bulk copy completing on an mbarrier (no tensor map, no multicast)
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+// shared -> global bulk copy in a bulk async-group
+__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Barrier that also returns the OR of `pred` over the participating threads.
+__device__ __forceinline__ int bar_red_or(int id, int n, int pred) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred), "r"(id), "r"(n)
+        : "memory");
+    return r;
+}
+
+// ----------------------------------------------------------------------------
+// Thread tile: a 256-thread group holds 128/d units; each unit's d x d state is
+// spread over 2d threads as 8 row groups x (d/4) column groups.  A thread owns
+// rows [r0, r0 + d/8) and columns [4*cg, 4*cg + 4).  The d/4 threads of a row
+// group are consecutive lanes of one warp.
+// ----------------------------------------------------------------------------
+template <int D>
+struct Geo {
+    static constexpr int RPT = D / 8;     // rows per thread
+    static constexpr int LPR = D / 4;     // lanes per row (column groups)
+    static constexpr int UPI = 128 / D;   // units per 256-thread group
+    static constexpr int TPU = 2 * D;     // threads per unit
+    static_assert(D == 16 || D == 32 || D == 64 || D == 128, "d in {16,32,64,128}");
+};
+
+// FP16-row bits of rows [r0, r0 + RPT) and the rank of row r0 among FP16 rows.
+// mask = the head's 128-bit FP16-row mask (bit i = key row i is FP16).
+template <int D>
+__device__ __forceinline__ void row_formats(uint4 mask, int r0, uint32_t& bits, int& rank16) {
+    constexpr int RPT = Geo<D>::RPT;
+    const int w = r0 >> 5, sh = r0 & 31;
+    const uint32_t word = (w == 0) ? mask.x : (w == 1) ? mask.y : (w == 2) ? mask.z : mask.w;
+    rank16 = (w > 0 ? __popc(mask.x) : 0) + (w > 1 ? __popc(mask.y) : 0) +
+             (w > 2 ? __popc(mask.z) : 0) + __popc(word & ((1u << sh) - 1u));
+    bits = (word >> sh) & ((1u << RPT) - 1u);
+}
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// Dequantize 4 INT8 codes (one 32-bit word) with an FP32 scale: fl(code*scale).
+// Codes are biased to 1..255 and placed in the mantissa of 2^23, so
+// (2^23 + c + 128) - (2^23 + 128) recovers c exactly without an I2F.
+__device__ __forceinline__ void dequant_int8x4(uint32_t w, float s, float2& lo, float2& hi) {
+    const uint32_t wb = w ^ 0x80808080u;
+    const float2 bias = f2(-8388736.0f);  // -(2^23 + 128)
+    float2 c01 = make_float2(__uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7440)),
+                             __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7441)));
+    float2 c23 = make_float2(__uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7442)),
+                             __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7443)));
+    c01 = __fadd2_rn(c01, bias);
+    c23 = __fadd2_rn(c23, bias);
+    lo = __fmul2_rn(c01, f2(s));
+    hi = __fmul2_rn(c23, f2(s));
+}
+
+__device__ __forceinline__ void dequant_fp16x4(uint2 h, float2& lo, float2& hi) {
+    lo = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    hi = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+}
+
+__device__ __forceinline__ uint2 quant_fp16x4(float2 lo, float2 hi) {
+    __half2 a = __float22half2_rn(lo);
+    __half2 b = __float22half2_rn(hi);
+    uint2 r;
+    r.x = *reinterpret_cast<uint32_t*>(&a);
+    r.y = *reinterpret_cast<uint32_t*>(&b);
+    return r;
+}
+
+// Codes of 4 values: RNE(x*inv).  fma(x, inv, 1.5*2^23) rounds the exact
+// product plus 1.5*2^23 once; |x*inv| <= 127 + 2^-16 keeps the sum inside
+// [2^23, 2^24) where the FP32 spacing is 1, so the rounding is to the nearest
+// integer with ties to even, and the low byte of the result's bit pattern is
+// the two's-complement code.  inv == 0 gives code 0.
+__device__ __forceinline__ uint32_t quant_int8x4(float2 lo, float2 hi, float inv) {
+    const float2 magic = f2(12582912.0f);
+    const float2 a = __ffma2_rn(lo, f2(inv), magic);
+    const float2 b = __ffma2_rn(hi, f2(inv), magic);
+    const uint32_t p01 = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040);
+    const uint32_t p23 = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040);
+    return __byte_perm(p01, p23, 0x5410);
+}
+
+__device__ __forceinline__ float absmax4(float2 lo, float2 hi) {
+    return fmaxf(fmaxf(fabsf(lo.x), fabsf(lo.y)), fmaxf(fabsf(hi.x), fabsf(hi.y)));
+}
+
+// Max over the d/4 lanes of a row group (all lanes get it).  d == 128 uses
+// one warp-wide integer max (|x| >= 0 orders like its bit pattern).
+template <int D>
+__device__ __forceinline__ float rowgroup_max(float m) {
+    if constexpr (D == 128) {
+        return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+    } else {
+#pragma unroll
+        for (int off = Geo<D>::LPR / 2; off >= 1; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        return m;
+    }
+}
+
+// scale = fl(a/127), inv = fl(127/a); zero / overflowing rows -> 0, 0.
+__device__ __forceinline__ void row_scale(float a, float& scale, float& inv) {
+    inv = __fdiv_rn(127.0f, a);
+    scale = __fdiv_rn(a, 127.0f);
+    if (a == 0.0f || isinf(inv)) {
+        inv = 0.0f;
+        scale = 0.0f;
+    }
+}
+
+// Load rows [r0, r0+RPT) x cols [4cg, 4cg+4) of a quantized block into x
+// (dequantized, not decayed).
+template <int D>
+__device__ __forceinline__ void load_quant_tile(const uint8_t* blk, uint32_t f16_off,
+                                                uint32_t i8_off, uint32_t bits, int rank16,
+                                                int r0, int cg, float2 (&x)[Geo<D>::RPT][2]) {
+    constexpr int RPT = Geo<D>::RPT;
+    int r16 = rank16, r8 = r0 - rank16;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        if ((bits >> i) & 1u) {
+            const uint2 h =
+                *reinterpret_cast<const uint2*>(blk + f16_off + (size_t)r16 * (2 * D) + cg * 8);
+            dequant_fp16x4(h, x[i][0], x[i][1]);
+            ++r16;
+        } else {
+            const uint32_t w =
+                *reinterpret_cast<const uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4);
+            const float s = *reinterpret_cast<const float*>(blk + (size_t)r8 * 4);
+            dequant_int8x4(w, s, x[i][0], x[i][1]);
+            ++r8;
+        }
+    }
+}
+
+// Requantize rows [r0, r0+RPT) of x into a quantized block at `blk` (shared or
+// global).  rowbuf: 2*RPT floats private to this row group (shared memory).
+// Must be called by every lane of the warp (it synchronises the warp).
+template <int D>
+__device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off, uint32_t i8_off,
+                                                 uint32_t bits, int rank16, int r0, int cg,
+                                                 const float2 (&x)[Geo<D>::RPT][2],
+                                                 float* rowbuf) {
+    constexpr int RPT = Geo<D>::RPT;
+    float amax[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        amax[i] = 0.0f;
+        if (D < 128 || !((bits >> i) & 1u)) amax[i] = rowgroup_max<D>(absmax4(x[i][0], x[i][1]));
+    }
+    // lane cg == 0 publishes the row maxima; lane cg < RPT takes row cg
+    if (cg == 0) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) rowbuf[i] = amax[i];
+    }
+    __syncwarp();
+    if (cg < RPT && !((bits >> cg) & 1u)) {
+        float scale, inv;
+        row_scale(rowbuf[cg], scale, inv);
+        rowbuf[RPT + cg] = inv;
+        const int rank8 = r0 + cg - rank16 - __popc(bits & ((1u << cg) - 1u));
+        *reinterpret_cast<float*>(blk + (size_t)rank8 * 4) = scale;
+    }
+    __syncwarp();
+    int r16 = rank16, r8 = r0 - rank16;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        if ((bits >> i) & 1u) {
+            *reinterpret_cast<uint2*>(blk + f16_off + (size_t)r16 * (2 * D) + cg * 8) =
+                quant_fp16x4(x[i][0], x[i][1]);
+            ++r16;
+        } else {
+            *reinterpret_cast<uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4) =
+                quant_int8x4(x[i][0], x[i][1], rowbuf[RPT + i]);
+            ++r8;
+        }
+    }
+    __syncwarp();  // rowbuf may be reused by the caller's next tile
+}
+
+}  // namespace damp

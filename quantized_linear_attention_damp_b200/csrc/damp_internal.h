@@ -1,0 +1,67 @@
+// damp_internal.h -- host/device shared definitions of libdamp (not installed).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace damp {
+
+// Header written at the start of the caller's pool buffer:
+//   [0, 16)                 device status word (uint32) + padding
+//   [16, 16 + 16*H)         per-head FP16-row masks, 4 x uint32 (key rows 0..127)
+// rounded up to 256 bytes; the blocks follow.
+constexpr size_t kStatusBytes = 16;
+constexpr int kMaskWords = 4;
+constexpr int kMaxD = 128;
+
+struct PoolDesc {
+    int format;      // DAMP_FMT_*
+    int n_slots, H, d, hp;
+    size_t block_bytes, block_stride, header_bytes, pool_bytes;
+    uint32_t f16_off, i8_off;  // byte offsets inside a quantized block
+    uint8_t* dev_buf;          // caller's buffer (NULL: host-only descriptor)
+    uint32_t* host_masks;      // [H][kMaskWords]
+};
+
+// Arguments of the decode-step kernel.
+struct StepArgs {
+    uint8_t* blocks;           // first block
+    const uint32_t* masks;     // [H][4]
+    uint32_t* status;
+    const int32_t* slot_idx;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    float* out;
+    int n, H, n_slots, hp;
+    uint32_t block_stride;     // bytes
+    uint32_t f16_off, i8_off;  // offsets inside a block
+    int n_items;               // work items (groups of 128/d units)
+    int n_stages;
+    // offsets inside one pipeline stage (bytes)
+    uint32_t stage_bytes, st_q, st_k, st_v, st_alpha, st_mask, st_meta;
+    uint32_t scratch_off;      // start of the consumers' reduction scratch
+    uint32_t bar_off;          // start of the mbarriers
+};
+
+// Arguments of the pack / unpack kernels.
+struct CodecArgs {
+    uint8_t* blocks;
+    const uint32_t* masks;
+    uint32_t* status;
+    const int32_t* slot_idx;
+    float* state;              // [n][H][d][d]
+    int n, H, n_slots, hp;
+    uint32_t block_stride, f16_off, i8_off;
+    int n_items;
+};
+
+// Launchers (damp_decode.cu, damp_codec.cu).  They return cudaError_t.
+cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
+                               cudaStream_t stream);
+cudaError_t launch_pack(const PoolDesc& p, const CodecArgs& a, cudaStream_t stream);
+cudaError_t launch_unpack(const PoolDesc& p, const CodecArgs& a, cudaStream_t stream);
+
+}  // namespace damp

@@ -1,0 +1,175 @@
+"""CPU checks of the C ABI: exported symbols, layout, host-side validation and
+block conversions.  No kernel is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import quantized_linear_attention_damp_b200 as D
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "damp.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(damp_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(D.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_has_the_same_names():
+    for n in declared_functions():
+        assert callable(getattr(D, n)), n
+
+
+def _golden():
+    vals = {}
+    for line in open(os.path.join(ROOT, "tests", "golden", "format_accounting.txt")):
+        line = line.split("#")[0].split()
+        if len(line) == 2:
+            vals[line[0]] = float(line[1])
+    return vals
+
+
+def test_format_accounting_matches_published_figures():
+    """27 FP16 rows + 101 INT8 rows + 101 FP32 scales at d = 128 give 9.885
+    bits/value (printed as 9.9) and 69.11 % less than FP32 (printed 69.1 %)."""
+    g = _golden()
+    d = int(g["d_k"])
+    block, stride = D.damp_layout(D.DAMP_FMT_MIXED, d, d, 27)
+    assert block == 20244 and stride == 20256
+    bits = block * 8 / (d * d)
+    assert round(bits, 1) == g["bits_per_value"]
+    assert round(100 * (1 - bits / 32), 1) == g["storage_reduction_percent"]
+    # 27 is the only FP16-row count that prints both figures
+    hits = []
+    for hp in range(0, d + 1):
+        b = D.damp_layout(D.DAMP_FMT_MIXED, d, d, hp)[0] * 8 / (d * d)
+        if round(b, 1) == g["bits_per_value"] and \
+                round(100 * (1 - b / 32), 1) == g["storage_reduction_percent"]:
+            hits.append(hp)
+    assert hits == [27]
+    # FP16 scales would not reproduce the figures (they give 9.8 bits)
+    b16 = (27 * d * 16 + 101 * d * 8 + 101 * 16) / (d * d)
+    assert round(b16, 1) != g["bits_per_value"]
+
+
+def test_layouts_of_other_formats():
+    assert D.damp_layout(D.DAMP_FMT_FP32, 128, 128, 0) == (65536, 65536)
+    assert D.damp_layout(D.DAMP_FMT_INT8_ROW, 128, 128, 0) == (16896, 16896)
+    assert D.damp_layout(D.DAMP_FMT_MIXED, 128, 128, 0) == (16896, 16896)
+    assert D.damp_layout(D.DAMP_FMT_MIXED, 128, 128, 128) == (32768, 32768)
+    assert D.damp_layout(D.DAMP_FMT_MIXED, 16, 16, 4) == (368, 368)
+    for d in (16, 32, 64, 128):
+        for hp in range(d + 1):
+            b, s = D.damp_layout(D.DAMP_FMT_MIXED, d, d, hp)
+            assert s % 16 == 0 and b <= s < b + 16 + 16
+
+
+def test_pool_bytes():
+    n = D.damp_pool_bytes(D.DAMP_FMT_MIXED, 64, 32, 128, 128, 27)
+    hdr = 256 * ((16 + 32 * 16 + 255) // 256)
+    assert n == hdr + 64 * 32 * 20256
+
+
+@pytest.mark.parametrize("args,status", [
+    ((3, 128, 128, 0), D.DAMP_ERR_INVALID_ARGUMENT),         # bad format
+    ((D.DAMP_FMT_MIXED, 128, 128, 129), D.DAMP_ERR_INVALID_ARGUMENT),
+    ((D.DAMP_FMT_MIXED, 128, 128, -1), D.DAMP_ERR_INVALID_ARGUMENT),
+    ((D.DAMP_FMT_INT8_ROW, 128, 128, 3), D.DAMP_ERR_INVALID_ARGUMENT),
+    ((D.DAMP_FMT_FP32, 128, 128, 1), D.DAMP_ERR_INVALID_ARGUMENT),
+    ((D.DAMP_FMT_MIXED, 128, 64, 0), D.DAMP_ERR_UNSUPPORTED),
+    ((D.DAMP_FMT_MIXED, 48, 48, 0), D.DAMP_ERR_UNSUPPORTED),
+    ((D.DAMP_FMT_MIXED, 256, 256, 0), D.DAMP_ERR_UNSUPPORTED),
+])
+def test_layout_rejects_bad_shapes(args, status):
+    with pytest.raises(D.DampError) as ei:
+        D.damp_layout(*args)
+    assert ei.value.status == status
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4, -5, -99):
+        assert isinstance(D.damp_status_string(s), str) and D.damp_status_string(s)
+
+
+def test_create_validates_the_fp16_row_map():
+    ok = np.array([[0, 5, 9], [1, 2, 3]])
+    h = D.damp_pool_create(D.DAMP_FMT_MIXED, 4, 2, 16, 16, 3, ok, None)
+    D.damp_pool_destroy(h)
+    for bad in (np.array([[0, 5, 5], [1, 2, 3]]), np.array([[0, 5, 16], [1, 2, 3]])):
+        with pytest.raises(D.DampError) as ei:
+            D.damp_pool_create(D.DAMP_FMT_MIXED, 4, 2, 16, 16, 3, bad, None)
+        assert ei.value.status == D.DAMP_ERR_INVALID_ARGUMENT
+    with pytest.raises(D.DampError):
+        D.damp_pool_create(D.DAMP_FMT_MIXED, 0, 2, 16, 16, 0, None, None)
+
+
+def test_create_checks_buffer_before_touching_the_device():
+    lib = ctypes.CDLL(D.LIB_PATH)
+    lib.damp_pool_create.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p, ctypes.c_void_p,
+                                                          ctypes.c_size_t,
+                                                          ctypes.POINTER(ctypes.c_void_p)]
+    out = ctypes.c_void_p()
+    need = D.damp_pool_bytes(D.DAMP_FMT_INT8_ROW, 2, 2, 16, 16, 0)
+    rc = lib.damp_pool_create(D.DAMP_FMT_INT8_ROW, 2, 2, 16, 16, 0, None, 0x10000, need - 1,
+                              ctypes.byref(out))
+    assert rc == D.DAMP_ERR_BUFFER_TOO_SMALL and not out.value
+    rc = lib.damp_pool_create(D.DAMP_FMT_INT8_ROW, 2, 2, 16, 16, 0, None, 0x10008, need,
+                              ctypes.byref(out))
+    assert rc == D.DAMP_ERR_MISALIGNED and not out.value
+
+
+def test_host_only_descriptor_rejects_device_calls():
+    h = D.damp_pool_create(D.DAMP_FMT_INT8_ROW, 2, 2, 16, 16, 0, None, None)
+    try:
+        lib = D._lib
+        assert lib.damp_decode_step(h, 1, 16, 0, 16, 16, 16, 0, 16, 16, 16, None) == \
+            D.DAMP_ERR_INVALID_ARGUMENT
+        assert lib.damp_pool_pack(h, 1, 16, 16, None) == D.DAMP_ERR_INVALID_ARGUMENT
+        assert lib.damp_decode_step(None, 1, 16, 0, 16, 16, 16, 0, 16, 16, 16, None) == \
+            D.DAMP_ERR_INVALID_ARGUMENT
+    finally:
+        D.damp_pool_destroy(h)
+
+
+@pytest.mark.parametrize("d,hp", [(16, 4), (64, 0), (128, 27), (128, 128)])
+def test_block_logical_round_trip(d, hp):
+    g = np.random.default_rng(d + hp)
+    H = 3
+    idx = np.stack([np.sort(g.permutation(d)[:hp]) for _ in range(H)])
+    h = D.damp_pool_create(D.DAMP_FMT_MIXED, 2, H, d, d, hp, idx if hp else None, None)
+    try:
+        _, stride = D.damp_layout(D.DAMP_FMT_MIXED, d, d, hp)
+        for head in range(H):
+            is16 = np.zeros(d, bool)
+            is16[idx[head]] = True
+            scale = np.where(is16, 0, g.uniform(0.1, 2, d)).astype(np.float32)
+            half = np.where(is16[:, None], g.integers(0, 0x7C00, (d, d)), 0).astype(np.uint16)
+            code = np.where(is16[:, None], 0, g.integers(-127, 128, (d, d))).astype(np.int8)
+            raw = D.damp_block_from_logical(h, head, stride, scale=scale, half=half, code=code)
+            assert raw.size == stride
+            back = D.damp_block_to_logical(h, head, raw, D.DAMP_FMT_MIXED, d)
+            assert np.array_equal(back["scale"], scale)
+            assert np.array_equal(back["half"], half)
+            assert np.array_equal(back["code"], code)
+            # byte order: scales of INT8 rows first, then FP16 rows, then INT8 rows
+            r = d - hp
+            assert np.array_equal(raw[:4 * r].view(np.float32), scale[~is16])
+            f16_off = (4 * r + 15) // 16 * 16
+            assert np.array_equal(raw[f16_off:f16_off + 2 * hp * d].view(np.uint16),
+                                  half[is16].reshape(-1))
+            assert np.array_equal(raw[f16_off + 2 * hp * d:f16_off + 2 * hp * d + r * d]
+                                  .view(np.int8), code[~is16].reshape(-1))
+    finally:
+        D.damp_pool_destroy(h)

@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA decode step (through the C ABI) against the oracle.
+
+Every test drives libdamp through its Python binding (C-ABI marshalling
+only) and the oracle from the same seeded inputs; each side keeps its own
+state.  States are expected bit-exact (each rounding is taken in the same
+precision and order on both sides); the asserted bar is the stated one:
+readouts within 1e-4 relative / 1e-5 absolute, FP16 rows and scales within
+1 ulp, INT8 codes within +-1 on at most 0.1 % of entries.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import quantized_linear_attention_damp_b200 as D
+import workloads as W
+from tests.gpu_helpers import Pair, torch_inputs
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # d=16, 1 slot x 2 heads, GDN, fp32 inputs, 4 FP16 rows/head (the tiny workload)
+    "tiny_gdn": W.WORKLOADS["tiny_gdn"],
+    # d=16 KDA, batch a strict subset of the pool (padding-free gather), 6 units:
+    # not a multiple of the 8 units a d=16 work item holds (ragged item)
+    "tiny_kda": W.Workload("tiny_kda", n=3, n_slots=4, H=2, d=16, hp=4, steps=8,
+                           gate=W.GATE_KDA, in_dtype="f32"),
+    "d32_gdn_bf16": W.Workload("d32_gdn_bf16", n=5, n_slots=6, H=3, d=32, hp=5, steps=4,
+                               gate=W.GATE_GDN, in_dtype="bf16"),
+    "d64_kda_bf16": W.Workload("d64_kda_bf16", n=7, n_slots=7, H=3, d=64, hp=13, steps=4,
+                               gate=W.GATE_KDA, in_dtype="bf16"),
+    # d=128 with a ragged tail: 37 x 5 = 185 units over ~296 resident CTAs
+    "d128_ragged": W.Workload("d128_ragged", n=37, n_slots=40, H=5, d=128, hp=27, steps=3,
+                              gate=W.GATE_GDN, in_dtype="bf16"),
+    "d128_kda_f32": W.Workload("d128_kda_f32", n=9, n_slots=9, H=4, d=128, hp=27, steps=3,
+                               gate=W.GATE_KDA, in_dtype="f32"),
+}
+
+
+def run_full(w, fmt, steps):
+    p = Pair(w, fmt)
+    try:
+        rep = p.check_state()
+        assert rep["exact"], rep            # pack parity
+        for s in range(steps):
+            x = W.step_inputs(w, s, p.hs)
+            out_g = p.gpu_step(x)
+            out_o = p.oracle_step_full(x)
+            p.check_out(out_g, out_o)
+            rep = p.check_state()
+            assert rep["exact"], (s, rep)
+        assert p.gpu.get_error() == 0
+    finally:
+        p.close()
+
+
+def test_tiny_gdn_full_trajectory():
+    """The tiny GDN workload: all 64 steps, whole state compared every step."""
+    w = W.WORKLOADS["tiny_gdn"]
+    run_full(w, "mixed", w.steps)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp32"])
+def test_small_shapes_all_formats(name, fmt):
+    w = SMALL[name]
+    run_full(w, fmt, min(w.steps, 8))
+
+
+@pytest.mark.parametrize("hp", [0, 1, 16])
+def test_tiny_extreme_fp16_row_counts(hp):
+    """No FP16 row, one FP16 row, every row FP16 (block without scales)."""
+    w = W.WORKLOADS["tiny_gdn"].with_(hp=hp, name=f"tiny_hp{hp}")
+    run_full(w, "mixed", 8)
+
+
+def test_all_fp16_rows_d128():
+    w = W.Workload("d128_allfp16", n=6, n_slots=6, H=2, d=128, hp=128, steps=3,
+                   gate=W.GATE_KDA, in_dtype="bf16")
+    run_full(w, "mixed", 3)
+
+
+@pytest.mark.parametrize("name,steps", [("gdn_batch", 3), ("kda", 2)])
+def test_full_size_whole_state(name, steps):
+    """The 64x32 GDN and 128x32 KDA workloads at full size, every unit compared."""
+    run_full(W.WORKLOADS[name], "mixed", steps)
+
+
+@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp32"])
+def test_high_concurrency_sampled_units(fmt):
+    """512 slots x 48 heads at full size (the launch the benchmark times);
+    sampled slots followed by the oracle over 4 steps."""
+    w = W.WORKLOADS["hiconc_gdn"]
+    slots = np.random.default_rng(5).choice(w.n_slots, 6, replace=False)
+    p = Pair(w, fmt, oracle_slots=slots)
+    try:
+        assert p.check_state()["exact"]
+        for s in range(4):
+            x = W.step_inputs(w, s, p.hs)
+            out_g = p.gpu_step(x)
+            out_o = p.oracle_step(x)
+            p.check_out(out_g, out_o)
+            assert p.check_state()["exact"], s
+        assert p.gpu.get_error() == 0
+    finally:
+        p.close()
+
+
+def test_long_trajectory_sampled_units():
+    """All 256 steps of the 64x32 GDN workload; 4 slots followed by the oracle."""
+    w = W.WORKLOADS["gdn_batch"]
+    p = Pair(w, "mixed", oracle_slots=[3, 17, 40, 63])
+    try:
+        for s in range(w.steps):
+            x = W.step_inputs(w, s, p.hs)
+            out_g = p.gpu_step(x)
+            p.check_out(out_g, p.oracle_step(x))
+            if s % 32 == 31:
+                assert p.check_state()["exact"], s
+        assert p.check_state()["exact"]
+    finally:
+        p.close()
+
+
+def test_padding_and_out_of_range_slots():
+    w = SMALL["d128_ragged"]
+    p = Pair(w, "mixed")
+    try:
+        x = W.step_inputs(w, 0, p.hs)
+        before = p.gpu.blocks().clone()
+        x.slot_idx[:] = -1
+        x.slot_idx[2] = 5
+        x.slot_idx[4] = w.n_slots + 3         # out of range: flagged, skipped
+        out_g = p.gpu_step(x)
+        assert not out_g[[0, 1, 3] + list(range(5, w.n))].any()
+        assert not out_g[4].any()
+        assert p.gpu.get_error(clear=True) == D.DAMP_EFLAG_SLOT_RANGE
+        assert p.gpu.get_error() == 0
+        after = p.gpu.blocks()
+        changed = (after != before).flatten(1).any(dim=1).view(w.n_slots, w.H)
+        assert changed[5].all() and changed.sum() == w.H
+        x.slot_idx[4] = -1
+        out_o = p.oracle_step_full(x)
+        p.check_out(out_g, out_o)
+        assert p.check_state()["exact"]
+    finally:
+        p.close()
+
+
+def test_identity_step_keeps_codes_on_gpu():
+    """alpha = 1, beta = 0 at full size: requantizing the dequantized state
+    leaves every code and FP16 value unchanged (scales within 1 ulp)."""
+    w = W.WORKLOADS["gdn_batch"]
+    p = Pair(w, "mixed", oracle_slots=[0])
+    try:
+        before = p.gpu.read_logical()
+        x = W.step_inputs(w, 0, p.hs)
+        x.alpha[:] = 1.0
+        x.beta[:] = 0.0
+        p.gpu_step(x)
+        after = p.gpu.read_logical()
+        assert np.array_equal(before["code"], after["code"])
+        assert np.array_equal(before["half"], after["half"])
+        ds = np.abs(before["scale"].view(np.int32).astype(np.int64)
+                    - after["scale"].view(np.int32))
+        assert ds.max() <= 1
+    finally:
+        p.close()
+
+
+def test_unpack_matches_oracle_reconstruction():
+    w = SMALL["d64_kda_bf16"]
+    p = Pair(w, "mixed")
+    try:
+        x = W.step_inputs(w, 0, p.hs)
+        p.gpu_step(x)
+        p.oracle_step_full(x)
+        out = torch.empty((w.n_slots, w.H, w.d, w.d), dtype=torch.float32, device="cuda")
+        p.gpu.unpack(torch.arange(w.n_slots, dtype=torch.int32, device="cuda"), out)
+        ref = O.unpack(p.ora, p.is_fp16[None])
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    finally:
+        p.close()
+
+
+def test_empty_batch_is_a_noop():
+    w = SMALL["tiny_kda"]
+    p = Pair(w, "mixed")
+    try:
+        before = p.gpu.blocks().clone()
+        e = torch.empty(0, dtype=torch.int32, device="cuda")
+        z = torch.empty((0, w.H, w.d), dtype=torch.float32, device="cuda")
+        a = torch.empty((0, w.H, w.d), dtype=torch.float32, device="cuda")
+        b = torch.empty((0, w.H), dtype=torch.float32, device="cuda")
+        p.gpu.step(e, z, z, z, a, b, z)
+        torch.cuda.synchronize()
+        assert torch.equal(before, p.gpu.blocks())
+    finally:
+        p.close()
+
+
+def test_argument_errors_enqueue_nothing():
+    w = SMALL["tiny_kda"]
+    p = Pair(w, "mixed")
+    try:
+        x = torch_inputs(w, W.step_inputs(w, 0, p.hs))
+        out = torch.empty((w.n, w.H, w.d), dtype=torch.float32, device="cuda")
+        before = p.gpu.blocks().clone()
+        mis = torch.empty(w.n * w.H * w.d + 1, dtype=torch.float32, device="cuda")[1:]
+        mis = mis.view(w.n, w.H, w.d)
+        with pytest.raises(D.DampError) as ei:
+            p.gpu.step(x["slot_idx"], mis, x["k"], x["v"], x["alpha"], x["beta"], out)
+        assert ei.value.status == D.DAMP_ERR_MISALIGNED
+        torch.cuda.synchronize()
+        assert torch.equal(before, p.gpu.blocks())
+    finally:
+        p.close()
