@@ -10,7 +10,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/damp.h"
+#include "damp.h"
 #include "damp_internal.h"
 
 using damp::PoolDesc;

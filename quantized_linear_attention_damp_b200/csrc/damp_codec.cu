@@ -16,7 +16,7 @@
 #include <algorithm>
 #include <mutex>
 
-#include "../../include/damp.h"
+#include "damp.h"
 #include "damp_device.cuh"
 
 namespace damp {

@@ -35,16 +35,15 @@
 #include <algorithm>
 #include <mutex>
 
-#include "../../include/damp.h"
+#include "damp.h"
 #include "damp_device.cuh"
 
 namespace damp {
 namespace {
 
-constexpr int kConsumerThreads = 256;
-constexpr int kThreads = 288;
+constexpr int kThreads = 256;
 
-struct Meta {  // one per unit in a stage, written by the producer
+struct Meta {  // one per unit in a stage, written by the issuing thread
     int slot;
     float alpha;  // GDN scalar decay
     float beta;
@@ -61,8 +60,13 @@ __device__ __forceinline__ float load_in(const uint8_t* base, int idx) {
     }
 }
 
+// bf16 value i of a packed pair-of-bf16 word array
+__device__ __forceinline__ float bf16_at(const uint32_t* w, int i) {
+    return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+}
+
 template <int D, bool QUANT, bool KDA, bool BF16>
-__global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs a) {
     using G = Geo<D>;
     constexpr int RPT = G::RPT, UPI = G::UPI, LPR = G::LPR;
     constexpr int LOGR = (RPT == 2) ? 1 : (RPT == 4) ? 2 : (RPT == 8) ? 3 : 4;
@@ -74,84 +78,94 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
     const int NS = a.n_stages;
     const uint32_t bar0 = smem_u32(smem + a.bar_off);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
-        }
+        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 1);
         fence_mbar_init();
     }
     __syncthreads();
 
     const int n_units = a.n * a.H;
+    const int my_items = (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int my_units = my_items * UPI;
 
-    // ------------------------------------------------------------------ producer
-    if (warp == 8) {
-        auto load_meta = [&](int item) {
-            Meta m{-1, 0.f, 0.f, 0};
-            const int u = item * UPI + lane;
-            if (lane < UPI && item < a.n_items && u < n_units) {
+    // ---- issue side (warp 0).  Lane L holds the metadata of CTA-local unit
+    // U == L (mod 32), loaded 32 units ahead of use, so the slot lookups never
+    // stall the pipeline.
+    auto load_meta = [&](int U) {
+        Meta m{-1, 0.f, 0.f, 0};
+        if (U < my_units) {
+            const int item = (int)blockIdx.x + (U / UPI) * (int)gridDim.x;
+            const int u = item * UPI + U % UPI;
+            if (u < n_units) {
                 m.exists = 1;
                 m.slot = __ldg(a.slot_idx + u / a.H);
                 if constexpr (!KDA) m.alpha = __ldg(a.alpha + u);
                 m.beta = __ldg(a.beta + u);
             }
-            return m;
-        };
-        int it = 0;
-        Meta cur = load_meta(blockIdx.x);
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x, ++it) {
-            const Meta nxt = load_meta(item + gridDim.x);  // prefetch one item ahead
-            const int stage = it % NS;
-            const uint32_t fill = static_cast<uint32_t>(it / NS);
-            bool ok = true;
-            if (fill > 0) ok = mbar_wait_bounded(empty_bar(stage), (fill - 1) & 1u);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
-                break;
-            }
-            uint8_t* st = smem + (size_t)stage * a.stage_bytes;
-            const int u = item * UPI + lane;
-            const bool load = cur.exists && cur.slot >= 0 && cur.slot < a.n_slots;
-            uint32_t tx = 0;
-            if (lane < UPI) {
-                *reinterpret_cast<Meta*>(st + a.st_meta + lane * sizeof(Meta)) = cur;
-                if (load) tx = a.block_stride + 3u * D * ELT + (KDA ? 4u * D : 0u) + 16u;
-            }
-            const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
-            __syncwarp();
-            if (lane == 0) {
-                if (tx_all) mbar_arrive_expect_tx(full_bar(stage), tx_all);
-                else mbar_arrive(full_bar(stage));
-            }
-            __syncwarp();
-            if (load) {
-                const int h = u % a.H;
-                const uint32_t fb = full_bar(stage);
-                const uint8_t* gblk =
-                    a.blocks + ((size_t)cur.slot * a.H + h) * (size_t)a.block_stride;
-                bulk_g2s(smem_u32(st + lane * a.block_stride), gblk, a.block_stride, fb);
-                const size_t io = (size_t)u * D * ELT;
-                bulk_g2s(smem_u32(st + a.st_q + lane * D * ELT),
-                         static_cast<const uint8_t*>(a.q) + io, D * ELT, fb);
-                bulk_g2s(smem_u32(st + a.st_k + lane * D * ELT),
-                         static_cast<const uint8_t*>(a.k) + io, D * ELT, fb);
-                bulk_g2s(smem_u32(st + a.st_v + lane * D * ELT),
-                         static_cast<const uint8_t*>(a.v) + io, D * ELT, fb);
-                if constexpr (KDA)
-                    bulk_g2s(smem_u32(st + a.st_alpha + lane * D * 4), a.alpha + (size_t)u * D,
-                             D * 4, fb);
-                bulk_g2s(smem_u32(st + a.st_mask + lane * 16), a.masks + (size_t)h * kMaskWords,
-                         16, fb);
-            }
-            cur = nxt;
         }
-        return;
-    }
+        return m;
+    };
+    Meta ring{-1, 0.f, 0.f, 0};
+    if (warp == 0) ring = load_meta(lane);
 
-    // ------------------------------------------------------------------ consumers
+    // Load work item `il` (CTA-local) into stage il % NS.  Warp 0 only.
+    auto issue = [&](int il) {
+        const int stage = il % NS;
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const int src = (il * UPI + lane) & 31;          // lane holding unit (il, lane)
+        Meta m;
+        m.slot = __shfl_sync(0xffffffffu, ring.slot, src);
+        m.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
+        m.beta = __shfl_sync(0xffffffffu, ring.beta, src);
+        m.exists = __shfl_sync(0xffffffffu, ring.exists, src);
+        // refill the ring entries consumed by this item
+        const int rel = (lane - il * UPI) & 31;
+        if (rel < UPI) ring = load_meta(il * UPI + rel + 32);
+        const bool load = lane < UPI && m.exists && m.slot >= 0 && m.slot < a.n_slots;
+        uint32_t tx = 0;
+        if (lane < UPI) {
+            *reinterpret_cast<Meta*>(st + a.st_meta + lane * sizeof(Meta)) = m;
+            if (load) tx = a.block_stride + 3u * D * ELT + (KDA ? 4u * D : 0u) + 16u;
+        }
+        const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
+        __syncwarp();
+        if (lane == 0) {
+            if (tx_all) mbar_arrive_expect_tx(full_bar(stage), tx_all);
+            else mbar_arrive(full_bar(stage));
+        }
+        __syncwarp();
+        if (load) {
+            const int item = (int)blockIdx.x + il * (int)gridDim.x;
+            const int u = item * UPI + lane;
+            const int h = u % a.H;
+            const uint32_t fb = full_bar(stage);
+            bulk_g2s(smem_u32(st + lane * a.block_stride),
+                     a.blocks + ((size_t)m.slot * a.H + h) * (size_t)a.block_stride,
+                     a.block_stride, fb);
+            const size_t io = (size_t)u * D * ELT;
+            bulk_g2s(smem_u32(st + a.st_q + lane * D * ELT), static_cast<const uint8_t*>(a.q) + io,
+                     D * ELT, fb);
+            bulk_g2s(smem_u32(st + a.st_k + lane * D * ELT), static_cast<const uint8_t*>(a.k) + io,
+                     D * ELT, fb);
+            bulk_g2s(smem_u32(st + a.st_v + lane * D * ELT), static_cast<const uint8_t*>(a.v) + io,
+                     D * ELT, fb);
+            if constexpr (KDA)
+                bulk_g2s(smem_u32(st + a.st_alpha + lane * D * 4), a.alpha + (size_t)u * D, D * 4,
+                         fb);
+            bulk_g2s(smem_u32(st + a.st_mask + lane * 16), a.masks + (size_t)h * kMaskWords, 16,
+                     fb);
+        }
+    };
+
+    // Stage of item il is refilled with item il + NS - 2 at the start of
+    // iteration il + ... : items il .. il + NS - 2 are in flight while item il
+    // is consumed; the stage of item il - 1 is still being stored.
+    const int ahead = NS - 2;
+    if (warp == 0)
+        for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
+
+    // ---- consumer side (all 8 warps)
     const int ui = tid / G::TPU;        // unit within the item
     const int tu = tid % G::TPU;        // thread within the unit
     const int cg = tu % LPR;            // column group: columns 4cg..4cg+3
@@ -167,7 +181,16 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
 
     int it = 0;
     bool aborted = false;
-    for (int item = blockIdx.x; item < a.n_items; item += gridDim.x, ++it) {
+    for (; it < my_items; ++it) {
+        const int item = (int)blockIdx.x + it * (int)gridDim.x;
+        if (warp == 0) {
+            const int il = it + ahead;
+            if (il < my_items) {
+                if (it >= 2 && lane == 0) bulk_wait_read<1>();  // store of item it-2 has read smem
+                __syncwarp();
+                issue(il);
+            }
+        }
         const int stage = it % NS;
         const uint32_t parity = static_cast<uint32_t>(it / NS) & 1u;
         const bool ok = mbar_wait_bounded(full_bar(stage), parity);
@@ -183,8 +206,17 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
         float2 x[RPT][2];
         uint32_t bits = 0;
         int rank16 = 0;
+        // k and q of this thread's rows (bf16 kept packed: two per word)
+        uint32_t kw[BF16 ? RPT / 2 : 1], qw[BF16 ? RPT / 2 : 1];
         if (active) {
-            // ---- step 1: reconstruct, then D_t S^
+            if constexpr (BF16) {
+#pragma unroll
+                for (int i = 0; i < RPT / 2; ++i) {
+                    kw[i] = reinterpret_cast<const uint32_t*>(sk)[r0 / 2 + i];
+                    qw[i] = reinterpret_cast<const uint32_t*>(sq)[r0 / 2 + i];
+                }
+            }
+            // ---- step 1: reconstruct S^
             if constexpr (QUANT) {
                 const uint4 mw = *reinterpret_cast<const uint4*>(st + a.st_mask + ui * 16);
                 row_formats<D>(mw, r0, bits, rank16);
@@ -198,21 +230,28 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
                     x[i][1] = make_float2(f.z, f.w);
                 }
             }
-            // ---- step 2 (first half): u = k^T S' (pairwise), w = q^T S', c = q^T (beta k)
+            // ---- step 2 (first half): S' = D S^; u = k^T S' (pairwise); w = q^T S'
             float2 stk[LOGR][2];
             float2 usum0 = f2(0.f), usum1 = f2(0.f);
             float2 w0 = f2(0.f), w1 = f2(0.f);
-            float cp = 0.f;
 #pragma unroll
             for (int i = 0; i < RPT; ++i) {
                 const int r = r0 + i;
                 const float al = KDA ? salpha[r] : meta.alpha;
                 x[i][0] = __fmul2_rn(x[i][0], f2(al));
                 x[i][1] = __fmul2_rn(x[i][1], f2(al));
-                const float kr = load_in<BF16>(sk, r);
-                const float qr = load_in<BF16>(sq, r);
-                float2 v0 = __fmul2_rn(f2(kr), x[i][0]);
-                float2 v1 = __fmul2_rn(f2(kr), x[i][1]);
+                float kr, qr;
+                if constexpr (BF16) {
+                    kr = bf16_at(kw, i);
+                    qr = bf16_at(qw, i);
+                } else {
+                    kr = load_in<false>(sk, r);
+                    qr = load_in<false>(sq, r);
+                }
+                // leaf products rounded on their own (scalar multiplies: never
+                // fused with the pairwise additions that follow)
+                float2 v0 = mul2_rn(f2(kr), x[i][0]);
+                float2 v1 = mul2_rn(f2(kr), x[i][1]);
 #pragma unroll
                 for (int b = 0; b < LOGR; ++b) {
                     if ((i >> b) & 1) {
@@ -230,15 +269,23 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
                 }
                 w0 = __ffma2_rn(f2(qr), x[i][0], w0);
                 w1 = __ffma2_rn(f2(qr), x[i][1], w1);
-                cp = __fmaf_rn(qr, __fmul_rn(meta.beta, kr), cp);
             }
             float* ru = red_u + (ui * 8 + rg) * D + 4 * cg;
             float* rw = red_w + (ui * 8 + rg) * D + 4 * cg;
             *reinterpret_cast<float4*>(ru) = make_float4(usum0.x, usum0.y, usum1.x, usum1.y);
             *reinterpret_cast<float4*>(rw) = make_float4(w0.x, w0.y, w1.x, w1.y);
+            // c = q^T (beta k) over this row group: lane cg < RPT takes row r0 + cg
+            float cp = 0.f;
+            if (cg < RPT) {
+                const float kr = load_in<BF16>(sk, r0 + cg), qr = load_in<BF16>(sq, r0 + cg);
+                cp = __fmul_rn(qr, __fmul_rn(meta.beta, kr));
+            }
+#pragma unroll
+            for (int off = LPR / 2; off >= 1; off >>= 1)
+                cp += __shfl_xor_sync(0xffffffffu, cp, off);
             if (cg == 0) cpart_s[ui * 8 + rg] = cp;
         }
-        if (bar_red_or(1, kConsumerThreads, ok ? 0 : 1)) {
+        if (bar_red_or(0, kThreads, ok ? 0 : 1)) {
             aborted = true;
             break;
         }
@@ -268,7 +315,7 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
                 if (j == 0 && meta.slot >= a.n_slots) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
             }
         }
-        bar_sync(1, kConsumerThreads);
+        __syncthreads();
 
         // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
         if (active) {
@@ -276,7 +323,8 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
             const float2 d0 = make_float2(dl.x, dl.y), d1 = make_float2(dl.z, dl.w);
 #pragma unroll
             for (int i = 0; i < RPT; ++i) {
-                const float b = __fmul_rn(meta.beta, load_in<BF16>(sk, r0 + i));
+                const float kr = BF16 ? bf16_at(kw, i) : load_in<BF16>(sk, r0 + i);
+                const float b = __fmul_rn(meta.beta, kr);
                 x[i][0] = __ffma2_rn(f2(b), d0, x[i][0]);
                 x[i][1] = __ffma2_rn(f2(b), d1, x[i][1]);
             }
@@ -290,9 +338,9 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
             }
             fence_proxy_async_smem();
         }
-        bar_sync(1, kConsumerThreads);
+        __syncthreads();
 
-        // ---- write back and recycle the previous stage
+        // ---- write back (one bulk store per block)
         if (tid == 0) {
 #pragma unroll
             for (int w = 0; w < UPI; ++w) {
@@ -305,21 +353,16 @@ __global__ void __maxnreg__(112) decode_step_kernel(const StepArgs a) {
                 }
             }
             bulk_commit();
-            if (it > 0) {
-                bulk_wait_read<1>();
-                mbar_arrive(empty_bar((it - 1) % NS));
-            }
         }
     }
 
     if (tid == 0) {
         if (aborted) {
             atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
-            // drain copies that may still be landing in this CTA's stages
-            for (int j = 0; j < NS; ++j) {
+            // drain loads that may still be landing in this CTA's stages
+            for (int j = 0; j <= ahead; ++j) {
                 const int jt = it + j;
-                const int item = blockIdx.x + jt * gridDim.x;
-                if (item >= a.n_items) break;
+                if (jt >= my_items) break;
                 (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
                                         100000000ull);
             }
@@ -396,7 +439,7 @@ cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
     };
     uint32_t ns = stages_for(per_cta_2);
     if (ns < 3) ns = stages_for(per_cta_1);
-    if (ns < 2) return cudaErrorInvalidConfiguration;
+    if (ns < 3) return cudaErrorInvalidConfiguration;
     a.n_stages = static_cast<int>(ns);
     a.stage_bytes = L.stage_bytes;
     a.st_q = L.st_q;
@@ -407,7 +450,7 @@ cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
     a.st_meta = L.st_meta;
     a.scratch_off = ns * L.stage_bytes;
     a.bar_off = a.scratch_off + L.scratch_bytes;
-    const size_t smem = a.bar_off + 16u * ns;
+    const size_t smem = a.bar_off + 8u * ns;
     int per_sm = 0;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) !=
         cudaSuccess)

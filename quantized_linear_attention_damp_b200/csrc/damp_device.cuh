@@ -145,6 +145,14 @@ __device__ __forceinline__ void row_formats(uint4 mask, int r0, uint32_t& bits, 
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
+// Two FP32 products, each rounded to nearest even.  Written as two scalar
+// multiplies: on sm_100a the packed f32x2 multiply did not reproduce the
+// scalar round-to-nearest product for every operand pair, and every product
+// here feeds a stored, bit-exact value.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+}
+
 // Dequantize 4 INT8 codes (one 32-bit word) with an FP32 scale: fl(code*scale).
 // Codes are biased to 1..255 and placed in the mantissa of 2^23, so
 // (2^23 + c + 128) - (2^23 + 128) recovers c exactly without an I2F.
@@ -157,8 +165,8 @@ __device__ __forceinline__ void dequant_int8x4(uint32_t w, float s, float2& lo, 
                              __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7443)));
     c01 = __fadd2_rn(c01, bias);
     c23 = __fadd2_rn(c23, bias);
-    lo = __fmul2_rn(c01, f2(s));
-    hi = __fmul2_rn(c23, f2(s));
+    lo = mul2_rn(c01, f2(s));
+    hi = mul2_rn(c23, f2(s));
 }
 
 __device__ __forceinline__ void dequant_fp16x4(uint2 h, float2& lo, float2& hi) {
