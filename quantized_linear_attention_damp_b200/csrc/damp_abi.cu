@@ -52,7 +52,7 @@ void layout(int format, int d, int hp, size_t* bytes, size_t* stride, uint32_t* 
 }
 
 size_t header_bytes(int H) {
-    return align_up(damp::kStatusBytes + (size_t)H * damp::kMaskWords * 4, 256);
+    return align_up(damp::dir_offset(H) + (size_t)H * damp::kDirWords * 4, 256);
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? DAMP_OK : DAMP_ERR_CUDA; }
@@ -127,6 +127,7 @@ int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_ro
     d.hp = hp_rows;
     layout(format, d_k, hp_rows, &d.block_bytes, &d.block_stride, &d.f16_off, &d.i8_off);
     d.header_bytes = header_bytes(H);
+    d.dir_off = damp::dir_offset(H);
     d.pool_bytes = d.header_bytes + (size_t)n_slots * H * d.block_stride;
     if (dev_buf) {
         if (!aligned16(dev_buf)) return DAMP_ERR_MISALIGNED;
@@ -145,6 +146,25 @@ int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_ro
     if (dev_buf) {
         std::vector<uint8_t> hdr(d.header_bytes, 0);
         memcpy(hdr.data() + damp::kStatusBytes, masks.data(), masks.size() * 4);
+        if (format != DAMP_FMT_FP32) {
+            // row directory: offsets of each key row (and its scale) in a block
+            uint32_t* dir = reinterpret_cast<uint32_t*>(hdr.data() + d.dir_off);
+            for (int h = 0; h < H; ++h) {
+                uint32_t r16 = 0, r8 = 0;
+                for (int i = 0; i < d_k; ++i) {
+                    const bool f16 = (masks[(size_t)h * damp::kMaskWords + (i >> 5)] >> (i & 31)) & 1u;
+                    uint32_t e;
+                    if (f16) {
+                        e = (d.f16_off + r16 * 2u * d_k) | (1u << 31);
+                        ++r16;
+                    } else {
+                        e = (d.i8_off + r8 * (uint32_t)d_k) | ((4u * r8) << 16);
+                        ++r8;
+                    }
+                    dir[(size_t)h * damp::kDirWords + i] = e;
+                }
+            }
+        }
         const cudaError_t e = cudaMemcpy(dev_buf, hdr.data(), hdr.size(), cudaMemcpyHostToDevice);
         if (e != cudaSuccess) {
             delete[] p->d.host_masks;
@@ -233,6 +253,7 @@ int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int 
     damp::StepArgs a{};
     a.blocks = d.dev_buf + d.header_bytes;
     a.masks = reinterpret_cast<const uint32_t*>(d.dev_buf + damp::kStatusBytes);
+    a.dir = reinterpret_cast<const uint32_t*>(d.dev_buf + d.dir_off);
     a.status = reinterpret_cast<uint32_t*>(d.dev_buf);
     a.slot_idx = slot_idx;
     a.q = q;

@@ -106,10 +106,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         }
         return m;
     };
+    constexpr int kIssueWarp = kThreads / 32 - 1;   // idle while columns are combined
     Meta ring{-1, 0.f, 0.f, 0};
-    if (warp == 0) ring = load_meta(lane);
+    if (warp == kIssueWarp) ring = load_meta(lane);
 
-    // Load work item `il` (CTA-local) into stage il % NS.  Warp 0 only.
+    // Load work item `il` (CTA-local) into stage il % NS.  Issue warp only.
     auto issue = [&](int il) {
         const int stage = il % NS;
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         uint32_t tx = 0;
         if (lane < UPI) {
             *reinterpret_cast<Meta*>(st + a.st_meta + lane * sizeof(Meta)) = m;
-            if (load) tx = a.block_stride + 3u * D * ELT + (KDA ? 4u * D : 0u) + 16u;
+            if (load) tx = a.block_stride + 3u * D * ELT + (KDA ? 4u * D : 0u) + (QUANT ? 4u * D : 0u);
         }
         const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
         __syncwarp();
@@ -153,8 +154,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             if constexpr (KDA)
                 bulk_g2s(smem_u32(st + a.st_alpha + lane * D * 4), a.alpha + (size_t)u * D, D * 4,
                          fb);
-            bulk_g2s(smem_u32(st + a.st_mask + lane * 16), a.masks + (size_t)h * kMaskWords, 16,
-                     fb);
+            if constexpr (QUANT)
+                bulk_g2s(smem_u32(st + a.st_dir + lane * D * 4), a.dir + (size_t)h * kDirWords,
+                         D * 4, fb);
         }
     };
 
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
     // iteration il + ... : items il .. il + NS - 2 are in flight while item il
     // is consumed; the stage of item il - 1 is still being stored.
     const int ahead = NS - 2;
-    if (warp == 0)
+    if (warp == kIssueWarp)
         for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
 
     // ---- consumer side (all 8 warps)
@@ -183,14 +185,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
     bool aborted = false;
     for (; it < my_items; ++it) {
         const int item = (int)blockIdx.x + it * (int)gridDim.x;
-        if (warp == 0) {
-            const int il = it + ahead;
-            if (il < my_items) {
-                if (it >= 2 && lane == 0) bulk_wait_read<1>();  // store of item it-2 has read smem
-                __syncwarp();
-                issue(il);
-            }
-        }
         const int stage = it % NS;
         const uint32_t parity = static_cast<uint32_t>(it / NS) & 1u;
         const bool ok = mbar_wait_bounded(full_bar(stage), parity);
@@ -204,8 +198,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         const float* salpha = reinterpret_cast<const float*>(st + a.st_alpha) + ui * D;
 
         float2 x[RPT][2];
-        uint32_t bits = 0;
-        int rank16 = 0;
+        const uint32_t* sdir = reinterpret_cast<const uint32_t*>(st + a.st_dir) + ui * D;
         // k and q of this thread's rows (bf16 kept packed: two per word)
         uint32_t kw[BF16 ? RPT / 2 : 1], qw[BF16 ? RPT / 2 : 1];
         if (active) {
@@ -218,9 +211,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             }
             // ---- step 1: reconstruct S^
             if constexpr (QUANT) {
-                const uint4 mw = *reinterpret_cast<const uint4*>(st + a.st_mask + ui * 16);
-                row_formats<D>(mw, r0, bits, rank16);
-                load_quant_tile<D>(blk, a.f16_off, a.i8_off, bits, rank16, r0, cg, x);
+                load_tile_dir<D>(blk, sdir, r0, cg, x);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {
@@ -285,10 +276,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
                 cp += __shfl_xor_sync(0xffffffffu, cp, off);
             if (cg == 0) cpart_s[ui * 8 + rg] = cp;
         }
+        // the store of item it-2 (committed by thread 0) must have read its
+        // stage before the issue warp refills that stage below
+        if (tid == 0 && it >= 2) bulk_wait_read<1>();
         if (bar_red_or(0, kThreads, ok ? 0 : 1)) {
             aborted = true;
             break;
         }
+        if (warp == kIssueWarp && it + ahead < my_items) issue(it + ahead);
 
         // ---- step 2 (second half) + step 3: per column j, delta_j and out_j
         if (tu < D) {
@@ -329,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
                 x[i][1] = __ffma2_rn(f2(b), d1, x[i][1]);
             }
             if constexpr (QUANT) {
-                store_quant_tile<D>(blk, a.f16_off, a.i8_off, bits, rank16, r0, cg, x, rowbuf);
+                store_tile_dir<D>(blk, sdir, r0, cg, x, rowbuf);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i)
@@ -374,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
 // ---------------------------------------------------------------------- host
 
 struct Layout {
-    uint32_t stage_bytes, st_q, st_k, st_v, st_alpha, st_mask, st_meta;
+    uint32_t stage_bytes, st_q, st_k, st_v, st_alpha, st_mask, st_dir, st_meta;
     uint32_t scratch_bytes;
 };
 
@@ -392,8 +387,9 @@ Layout stage_layout(int d, uint32_t stride, int in_dtype, int gate) {
     off = align_up(off + upi * d * elt, 16);
     L.st_alpha = off;
     off += (gate == DAMP_GATE_VECTOR) ? upi * d * 4 : 0;
-    L.st_mask = off;
-    off += upi * 16;
+    L.st_mask = off;   // unused by the decode step (kept 0-sized)
+    L.st_dir = off;
+    off += upi * d * 4;
     L.st_meta = off;
     off += upi * sizeof(Meta);
     L.stage_bytes = align_up(off, 128);
@@ -447,6 +443,7 @@ cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
     a.st_v = L.st_v;
     a.st_alpha = L.st_alpha;
     a.st_mask = L.st_mask;
+    a.st_dir = L.st_dir;
     a.st_meta = L.st_meta;
     a.scratch_off = ns * L.stage_bytes;
     a.bar_off = a.scratch_off + L.scratch_bytes;

@@ -42,14 +42,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t tx)
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// try_wait with a suspend-time hint: a warp whose phase is not complete
+// sleeps (up to the hint) instead of spinning and taking issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -59,17 +61,19 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 // Every wait in the pipeline is bounded: after kWaitNs it gives up and the
-// caller records DAMP_EFLAG_TIMEOUT instead of spinning forever.
+// caller records DAMP_EFLAG_TIMEOUT instead of waiting forever.  The timer is
+// read once every 64 tries.
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    while (true) {
+    for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > limit_ns) return false;
+        if ((n & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
     }
 }
+
 // global -> shared bulk copy completing on an mbarrier (no tensor map, no multicast)
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
                                          uint32_t bar) {
@@ -293,6 +297,95 @@ __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off,
         }
     }
     __syncwarp();  // rowbuf may be reused by the caller's next tile
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory variants for the decode step, addressed through the head's
+// row directory (one word per key row: row offset, scale offset, FP16 flag).
+// The block sits in a pipeline stage followed by at least 256 more bytes of
+// the same allocation, so both candidate reads of a row (8 bytes as FP16, 4
+// bytes as INT8, plus the scale) are always in bounds and can be issued
+// unconditionally: no load waits on a branch, and the rows' dependency chains
+// overlap.  Stores are made per the row's format.
+// ---------------------------------------------------------------------------
+
+// fl(code * scale) for 4 INT8 codes, converting each byte directly.
+__device__ __forceinline__ void dequant_int8x4_cvt(uint32_t w, float s, float2& lo, float2& hi) {
+    const float2 c01 = make_float2((float)(int8_t)(w & 0xffu), (float)(int8_t)((w >> 8) & 0xffu));
+    const float2 c23 = make_float2((float)(int8_t)((w >> 16) & 0xffu), (float)(int8_t)(w >> 24));
+    lo = __fmul2_rn(c01, f2(s));
+    hi = __fmul2_rn(c23, f2(s));
+}
+
+// max(|a|, |b|, |c|, |d|) with a three-input maximum
+__device__ __forceinline__ float absmax4_3(float2 lo, float2 hi) {
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(fabsf(lo.x)), "f"(fabsf(lo.y)), "f"(fabsf(hi.x)));
+    return fmaxf(m, fabsf(hi.y));
+}
+
+template <int D>
+__device__ __forceinline__ void load_tile_dir(const uint8_t* blk, const uint32_t* dir, int r0,
+                                              int cg, float2 (&x)[Geo<D>::RPT][2]) {
+    constexpr int RPT = Geo<D>::RPT;
+    constexpr int BATCH = RPT < 8 ? RPT : 8;
+#pragma unroll
+    for (int i0 = 0; i0 < RPT; i0 += BATCH) {
+        uint32_t e[BATCH];
+        uint2 w16[BATCH];
+        uint32_t w8[BATCH];
+        float sc[BATCH];
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            e[j] = dir[r0 + i0 + j];
+            const uint8_t* row = blk + (e[j] & 0xffffu);
+            w16[j] = *reinterpret_cast<const uint2*>(row + cg * 8);
+            w8[j] = *reinterpret_cast<const uint32_t*>(row + cg * 4);
+            sc[j] = *reinterpret_cast<const float*>(blk + ((e[j] >> 16) & 0x7fffu));
+        }
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            if (e[j] >> 31) dequant_fp16x4(w16[j], x[i0 + j][0], x[i0 + j][1]);
+            else dequant_int8x4_cvt(w8[j], sc[j], x[i0 + j][0], x[i0 + j][1]);
+        }
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void store_tile_dir(uint8_t* blk, const uint32_t* dir, int r0, int cg,
+                                               const float2 (&x)[Geo<D>::RPT][2],
+                                               float* rowbuf) {
+    constexpr int RPT = Geo<D>::RPT;
+    float amax[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) amax[i] = rowgroup_max<D>(absmax4_3(x[i][0], x[i][1]));
+    if (cg == 0) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) rowbuf[i] = amax[i];
+    }
+    __syncwarp();
+    if (cg < RPT) {
+        const uint32_t e = dir[r0 + cg];
+        if (!(e >> 31)) {
+            float scale, inv;
+            row_scale(rowbuf[cg], scale, inv);
+            rowbuf[RPT + cg] = inv;
+            *reinterpret_cast<float*>(blk + ((e >> 16) & 0x7fffu)) = scale;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const uint32_t e = dir[r0 + i];
+        uint8_t* row = blk + (e & 0xffffu);
+        if (e >> 31) {
+            *reinterpret_cast<uint2*>(row + cg * 8) = quant_fp16x4(x[i][0], x[i][1]);
+        } else {
+            *reinterpret_cast<uint32_t*>(row + cg * 4) =
+                quant_int8x4(x[i][0], x[i][1], rowbuf[RPT + i]);
+        }
+    }
+    __syncwarp();
 }
 
 }  // namespace damp

@@ -7,12 +7,20 @@
 namespace damp {
 
 // Header written at the start of the caller's pool buffer:
-//   [0, 16)                 device status word (uint32) + padding
-//   [16, 16 + 16*H)         per-head FP16-row masks, 4 x uint32 (key rows 0..127)
+//   [0, 16)                      device status word (uint32) + padding
+//   [16, 16 + 16*H)              per-head FP16-row masks, 4 x uint32 (key rows 0..127)
+//   [dir_off, dir_off + 512*H)   per-head row directory, 128 x uint32 (see below)
 // rounded up to 256 bytes; the blocks follow.
+//
+// Row directory entry of key row i of a quantized block:
+//   bits  0..15  byte offset of the row inside the block
+//   bits 16..30  byte offset of the row's FP32 scale (INT8 rows; 0 for FP16 rows)
+//   bit  31      1 = FP16 row, 0 = INT8 row
 constexpr size_t kStatusBytes = 16;
 constexpr int kMaskWords = 4;
 constexpr int kMaxD = 128;
+constexpr int kDirWords = 128;
+inline size_t dir_offset(int H) { return (kStatusBytes + (size_t)H * kMaskWords * 4 + 15) / 16 * 16; }
 
 struct PoolDesc {
     int format;      // DAMP_FMT_*
@@ -21,12 +29,14 @@ struct PoolDesc {
     uint32_t f16_off, i8_off;  // byte offsets inside a quantized block
     uint8_t* dev_buf;          // caller's buffer (NULL: host-only descriptor)
     uint32_t* host_masks;      // [H][kMaskWords]
+    size_t dir_off;            // byte offset of the row directory in the header
 };
 
 // Arguments of the decode-step kernel.
 struct StepArgs {
     uint8_t* blocks;           // first block
     const uint32_t* masks;     // [H][4]
+    const uint32_t* dir;       // [H][128] row directory
     uint32_t* status;
     const int32_t* slot_idx;
     const void* q;
@@ -41,7 +51,7 @@ struct StepArgs {
     int n_items;               // work items (groups of 128/d units)
     int n_stages;
     // offsets inside one pipeline stage (bytes)
-    uint32_t stage_bytes, st_q, st_k, st_v, st_alpha, st_mask, st_meta;
+    uint32_t stage_bytes, st_q, st_k, st_v, st_alpha, st_mask, st_dir, st_meta;
     uint32_t scratch_off;      // start of the consumers' reduction scratch
     uint32_t bar_off;          // start of the mbarriers
 };

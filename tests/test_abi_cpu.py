@@ -78,7 +78,8 @@ def test_layouts_of_other_formats():
 
 def test_pool_bytes():
     n = D.damp_pool_bytes(D.DAMP_FMT_MIXED, 64, 32, 128, 128, 27)
-    hdr = 256 * ((16 + 32 * 16 + 255) // 256)
+    # status word, 16-byte FP16-row mask and 512-byte row directory per head
+    hdr = 256 * ((16 + 32 * 16 + 32 * 512 + 255) // 256)
     assert n == hdr + 64 * 32 * 20256
 
 
