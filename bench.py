@@ -6,8 +6,10 @@ A step is one decode step (dequantize, gated delta rule, readout,
 requantize in place) over every (slot, head) of the workload, i.e. one
 launch of the decode kernel.  The default workload is the 64-slot x 32-head
 GDN batch at d = 128 with 27 FP16 rows per head (9.885 bits/value).  Its state
-(41.5 MB) fits in L2, so a 256 MiB buffer is written before every timed step
-and only the step is timed (CUDA events on the launching stream, summed).
+(41.5 MB) fits in L2, so consecutive steps rotate over several pools and input
+sets totalling at least 4x L2 (every step reads cold state and pays for
+earlier write-backs); each step is timed with CUDA events on the launching
+stream and the durations are summed.
 
 Printed: one JSON line (rank 0).  `value` is head-steps/s over all ranks;
 `roofline` is the decode kernel's algorithmic bytes per launch over its mean
@@ -36,10 +38,9 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "head-steps/s and achieved HBM GB/s (% of B200 roofline) per decode step"
-FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["damp_decode.cu", "damp_device.cuh", "damp_internal.h"]
-PROFILE = os.path.join(ROOT, "profiles", "decode_step_gdn_batch_mixed.txt")
+PROFILE = os.path.join(ROOT, "profiles", "decode_step_hiconc_gdn_mixed.txt")
 
 
 # ---------------------------------------------------------------- accounting
@@ -156,10 +157,38 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def rank_workload(name: str, rank: int) -> W.Workload:
+    """The workload a rank steps: the same shape on every rank, its own slots
+    (a data-parallel shard of a larger serving pool: independent seed)."""
+    return W.WORKLOADS[name].with_(seed=rank)
+
+
+def max_over_ranks(seconds: float, world: int, device=None) -> float:
+    """Device time of a step sequence as the max over ranks (every rank calls)."""
+    if world <= 1:
+        return seconds
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- native arm
 
 class Bench:
-    def __init__(self, w: W.Workload, fmt: str, n_inputs: int, device):
+    """One workload on one GPU.
+
+    L2 handling: the steps rotate over enough pools (and input sets) that the
+    data a step touches is at least 4x the L2 size, so every timed step reads
+    its state from HBM and pays for the write-back of earlier steps, as a
+    serving pool much larger than L2 does.  No step is flushed or skipped.
+    """
+
+    def __init__(self, w: W.Workload, fmt: str, device, n_inputs: int | None = None):
         import torch
 
         import quantized_linear_attention_damp_b200 as D
@@ -167,15 +196,27 @@ class Bench:
         self.w, self.fmt, self.dev = w, fmt, device
         self.hs = W.head_structure(w.with_(fmt=fmt))
         hp = self.hs.hp_row_idx if fmt == "mixed" else None
-        self.pool = D.DampPool(fmt, w.n_slots, w.H, w.d, hp, device=device)
-        S0 = W.initial_state(w, range(w.n_slots))
-        self.pool.pack(torch.arange(w.n_slots, dtype=torch.int32, device=device),
-                       torch.from_numpy(S0).to(device))
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        _, stride = D.damp_layout(D.FORMATS[fmt], w.d, w.d, w.hp if fmt == "mixed" else 0)
+        state_bytes = w.n_slots * w.H * stride
+        self.n_pools = max(1, -(-4 * l2 // state_bytes))
+        S0 = torch.from_numpy(W.initial_state(w, range(w.n_slots))).to(device)
+        ident = torch.arange(w.n_slots, dtype=torch.int32, device=device)
+        self.pools = []
+        for _ in range(self.n_pools):
+            p = D.DampPool(fmt, w.n_slots, w.H, w.d, hp, device=device)
+            p.pack(ident, S0)
+            self.pools.append(p)
         del S0
-        self.host = [self._host_inputs(W.step_inputs(w, s, self.hs)) for s in range(n_inputs)]
+        x0 = self._host_inputs(W.step_inputs(w, 0, self.hs))
+        in_bytes = sum(v.numel() * v.element_size() for v in x0.values())
+        if n_inputs is None:
+            n_inputs = max(4, -(-2 * l2 // in_bytes))
+        self.host = [x0] + [self._host_inputs(W.step_inputs(w, s, self.hs))
+                            for s in range(1, n_inputs)]
         self.dev_in = [{k: v.to(device) for k, v in h.items()} for h in self.host]
         self.out = torch.empty((w.n, w.H, w.d), dtype=torch.float32, device=device)
-        self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.touched_bytes = self.n_pools * state_bytes
         torch.cuda.synchronize(device)
 
     def _host_inputs(self, x):
@@ -189,18 +230,15 @@ class Bench:
                  alpha=torch.from_numpy(x.alpha), beta=torch.from_numpy(x.beta))
         return {k: t.contiguous().pin_memory() for k, t in d.items()}
 
-    def flush(self):
-        self.flush_buf.zero_()
-
     def step(self, i: int):
         a = self.dev_in[i % len(self.dev_in)]
-        self.pool.step(a["slot_idx"], a["q"], a["k"], a["v"], a["alpha"], a["beta"], self.out)
+        self.pools[i % self.n_pools].step(a["slot_idx"], a["q"], a["k"], a["v"], a["alpha"],
+                                          a["beta"], self.out)
 
     def timed(self, steps: int, warmup: int, sampler=None) -> float:
-        """Seconds of device time over `steps` steps (L2 flushed before each)."""
+        """Seconds of device time over `steps` consecutive steps."""
         torch = self.torch
         for i in range(warmup):
-            self.flush()
             self.step(i)
         torch.cuda.synchronize(self.dev)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -208,7 +246,6 @@ class Bench:
         ctx = sampler if sampler is not None else _Null()
         with ctx:
             for i in range(steps):
-                self.flush()
                 ev[i][0].record()
                 self.step(warmup + i)
                 ev[i][1].record()
@@ -227,20 +264,21 @@ class Bench:
               for _ in range(steps)]
         torch.cuda.synchronize(self.dev)
         for i in range(steps):
-            self.flush()
             src = self.host[i % len(self.host)]
             ev[i][0].record()
             for k_, v_ in src.items():
                 dev_in[k_].copy_(v_, non_blocking=True)
-            self.pool.step(dev_in["slot_idx"], dev_in["q"], dev_in["k"], dev_in["v"],
-                           dev_in["alpha"], dev_in["beta"], self.out)
+            self.pools[i % self.n_pools].step(dev_in["slot_idx"], dev_in["q"], dev_in["k"],
+                                              dev_in["v"], dev_in["alpha"], dev_in["beta"],
+                                              self.out)
             out_host.copy_(self.out, non_blocking=True)
             ev[i][1].record()
         torch.cuda.synchronize(self.dev)
         return sum(a.elapsed_time(b) for a, b in ev) / 1e3, h2d, d2h
 
     def close(self):
-        self.pool.close()
+        for p in self.pools:
+            p.close()
 
 
 class _Null:
@@ -278,9 +316,9 @@ def run_native(args, rank, world, local_rank):
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = W.WORKLOADS[args.workload].with_(seed=rank)
+    w = rank_workload(args.workload, rank)
     fmt = args.fmt
-    b = Bench(w, fmt, n_inputs=16, device=dev)
+    b = Bench(w, fmt, device=dev)
     units = w.n * w.H
     ub = unit_bytes(w, fmt)
 
@@ -288,16 +326,11 @@ def run_native(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(local_rank)
-    secs = b.timed(args.steps, args.warmup, sampler)
+    secs = max_over_ranks(b.timed(args.steps, args.warmup, sampler), world, dev)
     if world > 1:
-        t = torch.tensor([secs], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        secs = float(t.item())
-    e2e_secs, h2d, d2h = b.timed_e2e(args.steps)
-    if world > 1:
-        t = torch.tensor([e2e_secs], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_secs = float(t.item())
+        dist.barrier()
+    e2e_secs, h2d, d2h = (b.timed_e2e(args.steps) if not args.no_e2e else (float("nan"), 0, 0))
+    e2e_secs = max_over_ranks(e2e_secs, world, dev)
     b.close()
 
     if rank != 0:
@@ -313,7 +346,8 @@ def run_native(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": describe(w, fmt), "units_per_step_per_gpu": units,
                    "algorithmic_bytes_per_unit": ub,
-                   "l2": "256 MiB buffer written before every timed step (state < L2)",
+                   "l2": f"steps rotate over {b.n_pools} pools ({b.touched_bytes / 1e6:.0f} MB) "
+                         "and their inputs, >= 4x L2: inputs larger than L2",
                    "timing": "CUDA events around each step on the launch stream, summed",
                    "parallelism": f"dp{world} (slots sharded, no collective)"},
         "hbm_gbs": gbs,
@@ -323,16 +357,17 @@ def run_native(args, rank, world, local_rank):
                      "traffic": profiled_traffic(units)},
         "gpu_launches": args.steps,
         "clocks": sampler.summary(),
-        "e2e": {"value": units * world * args.steps / e2e_secs, "unit": "head-steps/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": ({"value": units * world * args.steps / e2e_secs, "unit": "head-steps/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                if not args.no_e2e else None),
     }
-    if world == 1:
+    if world == 1 and args.cpu_seconds > 0:
         v, n, el = cpu_baseline(w, fmt, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "head-steps/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{n} (slot, head) units of {w.name} ({fmt}), "
                                           f"one step each, single thread, {el:.1f} s"}
-        if not args.no_variants:
-            line["variants"] = variants(args, dev)
+    if world == 1 and not args.no_variants:
+        line["variants"] = variants(args, dev)
     print(json.dumps(line), flush=True)
 
 
@@ -344,7 +379,7 @@ def variants(args, dev):
                       ("hiconc_gdn", "int8"), ("hiconc_gdn", "fp32"), ("gdn_batch", "int8"),
                       ("gdn_batch", "fp32")]:
         w = W.WORKLOADS[name]
-        b = Bench(w, fmt, n_inputs=4, device=dev)
+        b = Bench(w, fmt, device=dev)
         secs = b.timed(steps, 3)
         b.close()
         units = w.n * w.H
@@ -404,6 +439,7 @@ def main():
     ap.add_argument("--fmt", default="mixed", choices=["mixed", "int8", "fp32"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
