@@ -475,6 +475,11 @@ cudaError_t dispatch_fmt(const PoolDesc& p, const StepArgs& a, int in_dtype, int
 
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream) {
+    if (p.d == 128 && p.format != DAMP_FMT_FP32 && decode_pair_fits(a, in_dtype, gate)) {
+        StepArgs b = a;
+        b.n_items = ((a.n + 1) / 2) * a.H;   // pairs of batch entries x heads
+        return launch_decode_pair(b, in_dtype, gate, stream);
+    }
     switch (p.d) {
         case 16: return dispatch_fmt<16>(p, a, in_dtype, gate, stream);
         case 32: return dispatch_fmt<32>(p, a, in_dtype, gate, stream);

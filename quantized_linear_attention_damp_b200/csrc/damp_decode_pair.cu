@@ -1,0 +1,503 @@
+// damp_decode_pair.cu -- decode step for quantized d = 128 states, two units
+// of the same head per CTA iteration.
+//
+// Same arithmetic, same order of operations and same results as the generic
+// kernel in damp_decode.cu ("STEPQuant ...", Appendix Table C2 steps 1, 2,
+// 3, 6 on the DAMP row format); only the work decomposition differs.
+//
+// Why pairs.  A lane owns 8 columns of a row, so one row of one unit takes 16
+// lanes and a warp covers the same row of two units.  The two units are the
+// same head h of two batch entries, so they share the head's FP16-row map
+// and every row is FP16 or INT8 for the whole warp: format branches stay
+// warp-uniform while the per-row work (directory lookup, scale, k/q values,
+// row maximum, division, stores) is spread over 8 columns instead of 4.
+//
+// CTA of 16 warps: warp w owns key rows [8w, 8w + 8) of both units; lanes
+// 0-15 work on unit 0, lanes 16-31 on unit 1.  Each thread keeps its 8 x 8
+// tile in registers from dequantize to requantize.  u = k^T S' is summed in
+// the recursive pairwise order: 8 rows per thread as a subtree, then the top
+// four levels over the 16 row groups.  Warp 15, idle while columns are
+// combined, refills the pipeline (cp.async.bulk into a shared-memory ring of
+// stages completing on mbarriers, no tensor map, no multicast).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "damp.h"
+#include "damp_device.cuh"
+
+namespace damp {
+namespace {
+
+constexpr int kPT = 512;       // threads
+constexpr int kPD = 128;       // d_k = d_v
+constexpr int kPR = 8;         // rows per thread
+constexpr int kPG = 16;        // row groups (warps)
+
+// Per-unit metadata written by the issue warp into the stage (32 bytes).
+struct PMeta {
+    int active;        // 1: block loaded, to be updated and stored
+    int exists;        // 1: the pair has this batch entry (out row to write)
+    float alpha;       // GDN scalar decay
+    float beta;
+    long long unit;    // b*H + h: row of q/k/v/alpha/beta/out
+    long long boff;    // byte offset of the block in the pool; -1 if none
+};
+static_assert(sizeof(PMeta) == 32, "PMeta layout");
+
+template <bool BF16>
+__device__ __forceinline__ float in_at(const uint8_t* base, int idx) {
+    if constexpr (BF16) {
+        return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(base)[idx])
+                               << 16);
+    } else {
+        return reinterpret_cast<const float*>(base)[idx];
+    }
+}
+
+__device__ __forceinline__ float bf16w(const uint32_t* w, int i) {
+    return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+}
+
+// 8 INT8 codes (two words) times a scale, each product rounded once.
+__device__ __forceinline__ void dq_int8x8(uint2 w, float s, float2 (&x)[4]) {
+    dequant_int8x4_cvt(w.x, s, x[0], x[1]);
+    dequant_int8x4_cvt(w.y, s, x[2], x[3]);
+}
+__device__ __forceinline__ void dq_fp16x8(uint4 h, float2 (&x)[4]) {
+    dequant_fp16x4(make_uint2(h.x, h.y), x[0], x[1]);
+    dequant_fp16x4(make_uint2(h.z, h.w), x[2], x[3]);
+}
+__device__ __forceinline__ float absmax8(const float2 (&x)[4]) {
+    float m0, m1;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m0) : "f"(fabsf(x[0].x)), "f"(fabsf(x[0].y)), "f"(fabsf(x[1].x)));
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m1) : "f"(fabsf(x[1].y)), "f"(fabsf(x[2].x)), "f"(fabsf(x[2].y)));
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m0), "f"(m1), "f"(fabsf(x[3].x)));
+    return fmaxf(m, fabsf(x[3].y));
+}
+
+template <bool KDA, bool BF16>
+__global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
+    constexpr uint32_t ELT = BF16 ? 2 : 4;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int NS = a.n_stages;
+    const uint32_t bar0 = smem_u32(smem + a.bar_off);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int H = a.H;
+    const int my_items = (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int my_units = 2 * my_items;
+
+    // ---- issue side (warp 15): lane L holds the metadata of CTA-local unit
+    // U == L (mod 32), loaded 32 units ahead of use.
+    constexpr int kIssueWarp = kPT / 32 - 1;
+    auto load_meta = [&](int U) {
+        PMeta m{0, 0, 0.f, 0.f, 0, -1};
+        if (U < my_units) {
+            const int g = (int)blockIdx.x + (U >> 1) * (int)gridDim.x;  // item: pair p, head h
+            const int p = g / H, h = g - p * H;
+            const int b = 2 * p + (U & 1);
+            if (b < a.n) {
+                const long long u = (long long)b * H + h;
+                const int slot = __ldg(a.slot_idx + b);
+                m.exists = 1;
+                m.unit = u;
+                if constexpr (!KDA) m.alpha = __ldg(a.alpha + u);
+                m.beta = __ldg(a.beta + u);
+                if (slot >= 0 && slot < a.n_slots) {
+                    m.active = 1;
+                    m.boff = ((long long)slot * H + h) * (long long)a.block_stride;
+                } else if (slot >= a.n_slots) {
+                    m.active = -1;   // out of range: flagged by the consumer
+                }
+            }
+        }
+        return m;
+    };
+    PMeta ring{0, 0, 0.f, 0.f, 0, -1};
+    if (warp == kIssueWarp) ring = load_meta(lane);
+
+    auto issue = [&](int il) {
+        const int stage = il % NS;
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const int src = (2 * il + lane) & 31;
+        PMeta m;
+        m.active = __shfl_sync(0xffffffffu, ring.active, src);
+        m.exists = __shfl_sync(0xffffffffu, ring.exists, src);
+        m.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
+        m.beta = __shfl_sync(0xffffffffu, ring.beta, src);
+        m.unit = __shfl_sync(0xffffffffu, ring.unit, src);
+        m.boff = __shfl_sync(0xffffffffu, ring.boff, src);
+        const int rel = (lane - 2 * il) & 31;
+        if (rel < 2) ring = load_meta(2 * il + rel + 32);
+        const bool load = lane < 2 && m.active == 1;
+        const uint32_t loads = __ballot_sync(0xffffffffu, load);
+        uint32_t tx = 0;
+        if (lane < 2) {
+            *reinterpret_cast<PMeta*>(st + a.st_meta + lane * sizeof(PMeta)) = m;
+            if (load) tx = a.block_stride + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u);
+            if (lane == 0 && loads) tx += 4u * kPD;   // the head's row directory
+        }
+        const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
+        __syncwarp();
+        if (lane == 0) {
+            if (tx_all) mbar_arrive_expect_tx(full_bar(stage), tx_all);
+            else mbar_arrive(full_bar(stage));
+        }
+        __syncwarp();
+        const uint32_t fb = full_bar(stage);
+        if (load) {
+            bulk_g2s(smem_u32(st + lane * a.block_stride), a.blocks + m.boff, a.block_stride, fb);
+            const size_t io = (size_t)m.unit * kPD * ELT;
+            bulk_g2s(smem_u32(st + a.st_q + lane * kPD * ELT),
+                     static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
+            bulk_g2s(smem_u32(st + a.st_k + lane * kPD * ELT),
+                     static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
+            bulk_g2s(smem_u32(st + a.st_v + lane * kPD * ELT),
+                     static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
+            if constexpr (KDA)
+                bulk_g2s(smem_u32(st + a.st_alpha + lane * kPD * 4), a.alpha + (size_t)m.unit * kPD,
+                         kPD * 4, fb);
+        }
+        if (loads) {
+            // both units of the item share head h = unit mod H
+            const int hl = __ffs(loads) - 1;
+            const long long uu = __shfl_sync(0xffffffffu, m.unit, hl);
+            if (lane == 0)
+                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)(uu % H) * kDirWords, kPD * 4, fb);
+        }
+    };
+
+    const int ahead = NS - 2;
+    if (warp == kIssueWarp)
+        for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
+
+    // ---- consumers
+    const int ui = lane >> 4;           // unit of the pair
+    const int cg = lane & 15;           // columns 8cg .. 8cg+7
+    const int r0 = warp * kPR;          // rows r0 .. r0+7
+
+    uint8_t* scratch = smem + a.scratch_off;
+    float* red_u = reinterpret_cast<float*>(scratch);            // [2][16][128]
+    float* red_w = red_u + 2 * kPG * kPD;                        // [2][16][128]
+    float* delta_s = red_w + 2 * kPG * kPD;                      // [2][128]
+    float* cpart_s = delta_s + 2 * kPD;                          // [2][16]
+    float* rowbuf = cpart_s + 2 * kPG + (warp * 2 + ui) * 16;    // this half-warp's 16 floats
+
+    int it = 0, stage = 0;
+    uint32_t parity = 0;
+    bool aborted = false;
+    for (; it < my_items; ++it) {
+        const bool ok = mbar_wait_bounded(full_bar(stage), parity);
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const PMeta meta = *reinterpret_cast<const PMeta*>(st + a.st_meta + ui * sizeof(PMeta));
+        const PMeta mo = *reinterpret_cast<const PMeta*>(st + a.st_meta + (ui ^ 1) * sizeof(PMeta));
+        // The directory (and so every row offset) is valid only if at least one
+        // unit of the item was loaded; this is uniform over the CTA.
+        const bool any = ok && (meta.active == 1 || mo.active == 1);
+        uint8_t* blk = st + ui * a.block_stride;
+        const uint8_t* sq = st + a.st_q + ui * kPD * ELT;
+        const uint8_t* sk = st + a.st_k + ui * kPD * ELT;
+        const float* salpha = reinterpret_cast<const float*>(st + a.st_alpha) + ui * kPD;
+        const uint32_t* sdir = reinterpret_cast<const uint32_t*>(st + a.st_dir) + r0;
+        const uint8_t* b16 = blk + cg * 16;   // this lane's 16 bytes of an FP16 row
+        const uint8_t* b8 = blk + cg * 8;     // this lane's 8 bytes of an INT8 row
+
+        // Every lane computes (an inactive half works on stale stage data
+        // and skips every global side effect), so warp-level operations
+        // always see a full warp.
+        float2 x[kPR][4];
+        uint32_t kw[BF16 ? kPR / 2 : 1], qw[BF16 ? kPR / 2 : 1];
+        auto kval = [&](int i) { return BF16 ? bf16w(kw, i) : in_at<false>(sk, r0 + i); };
+        auto qval = [&](int i) { return BF16 ? bf16w(qw, i) : in_at<false>(sq, r0 + i); };
+        uint32_t dir[kPR];
+        if (any) {
+            if constexpr (BF16) {
+                const uint4 kv = *reinterpret_cast<const uint4*>(sk + 2 * r0);
+                const uint4 qv = *reinterpret_cast<const uint4*>(sq + 2 * r0);
+                kw[0] = kv.x; kw[1] = kv.y; kw[2] = kv.z; kw[3] = kv.w;
+                qw[0] = qv.x; qw[1] = qv.y; qw[2] = qv.z; qw[3] = qv.w;
+            }
+            {
+                const uint4 d0 = reinterpret_cast<const uint4*>(sdir)[0];
+                const uint4 d1 = reinterpret_cast<const uint4*>(sdir)[1];
+                dir[0] = d0.x; dir[1] = d0.y; dir[2] = d0.z; dir[3] = d0.w;
+                dir[4] = d1.x; dir[5] = d1.y; dir[6] = d1.z; dir[7] = d1.w;
+            }
+            // ---- step 1: reconstruct S^ (all candidate reads first, then decode)
+#pragma unroll
+            for (int i0 = 0; i0 < kPR; i0 += 4) {
+                uint4 w16[4];
+                uint2 w8[4];
+                float sc[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t e = dir[i0 + j], off = e & 0xffffu;
+                    w16[j] = *reinterpret_cast<const uint4*>(b16 + off);
+                    w8[j] = *reinterpret_cast<const uint2*>(b8 + off);
+                    sc[j] = *reinterpret_cast<const float*>(blk + ((e >> 16) & 0x7fffu));
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (dir[i0 + j] >> 31) dq_fp16x8(w16[j], x[i0 + j]);
+                    else dq_int8x8(w8[j], sc[j], x[i0 + j]);
+                }
+            }
+            // ---- step 2 (first half): S' = D S^; u = k^T S' (pairwise); w = q^T S'
+            float2 stk[3][4];
+            float2 us[4], ws[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ws[c] = f2(0.f);
+#pragma unroll
+            for (int i = 0; i < kPR; ++i) {
+                const float al = KDA ? salpha[r0 + i] : meta.alpha;
+                const float kr = kval(i), qr = qval(i);
+                float2 v[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    x[i][c] = __fmul2_rn(x[i][c], f2(al));
+                    v[c] = mul2_rn(f2(kr), x[i][c]);      // scalar products: never fused
+                    ws[c] = __ffma2_rn(f2(qr), x[i][c], ws[c]);
+                }
+#pragma unroll
+                for (int lv = 0; lv < 3; ++lv) {
+                    if ((i >> lv) & 1) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) v[c] = __fadd2_rn(stk[lv][c], v[c]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) stk[lv][c] = v[c];
+                        break;
+                    }
+                }
+                if (i == kPR - 1) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) us[c] = v[c];
+                }
+            }
+            float* ru = red_u + (ui * kPG + warp) * kPD + 8 * cg;
+            float* rw = red_w + (ui * kPG + warp) * kPD + 8 * cg;
+            reinterpret_cast<float4*>(ru)[0] = make_float4(us[0].x, us[0].y, us[1].x, us[1].y);
+            reinterpret_cast<float4*>(ru)[1] = make_float4(us[2].x, us[2].y, us[3].x, us[3].y);
+            reinterpret_cast<float4*>(rw)[0] = make_float4(ws[0].x, ws[0].y, ws[1].x, ws[1].y);
+            reinterpret_cast<float4*>(rw)[1] = make_float4(ws[2].x, ws[2].y, ws[3].x, ws[3].y);
+            // c = q^T (beta k) over this row group: lane cg < 8 takes row r0 + cg
+            float cp = 0.f;
+            if (cg < kPR) cp = __fmul_rn(in_at<BF16>(sq, r0 + cg),
+                                         __fmul_rn(meta.beta, in_at<BF16>(sk, r0 + cg)));
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
+            if (cg == 0) cpart_s[ui * kPG + warp] = cp;
+        }
+        if (tid == 0 && it >= 2) bulk_wait_read<1>();   // store of item it-2 has read its stage
+        if (bar_red_or(0, kPT, ok ? 0 : 1)) {
+            aborted = true;
+            break;
+        }
+
+        // ---- step 2 (second half) + step 3: delta_j and out_j, 2 x 128 columns
+        if (warp == kIssueWarp && it + ahead < my_items) issue(it + ahead);
+        if (tid < 2 * kPD) {
+            const int cu_ = tid >> 7, j = tid & (kPD - 1);
+            const PMeta m = *reinterpret_cast<const PMeta*>(st + a.st_meta + cu_ * sizeof(PMeta));
+            if (m.active == 1) {
+                const float* c0 = red_u + cu_ * kPG * kPD + j;
+                float t[8];
+#pragma unroll
+                for (int q2 = 0; q2 < 8; ++q2)
+                    t[q2] = __fadd_rn(c0[(2 * q2) * kPD], c0[(2 * q2 + 1) * kPD]);
+                const float uj = __fadd_rn(
+                    __fadd_rn(__fadd_rn(t[0], t[1]), __fadd_rn(t[2], t[3])),
+                    __fadd_rn(__fadd_rn(t[4], t[5]), __fadd_rn(t[6], t[7])));
+                const float* w0 = red_w + cu_ * kPG * kPD + j;
+                float wj = 0.f;
+#pragma unroll
+                for (int q2 = 0; q2 < kPG; ++q2) wj = __fadd_rn(wj, w0[q2 * kPD]);
+                const float4* cpp = reinterpret_cast<const float4*>(cpart_s + cu_ * kPG);
+                float c = 0.f;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 v4 = cpp[q4];
+                    c += (v4.x + v4.y) + (v4.z + v4.w);
+                }
+                const float vj = in_at<BF16>(st + a.st_v + cu_ * kPD * ELT, j);
+                const float dj = __fsub_rn(vj, uj);
+                delta_s[cu_ * kPD + j] = dj;
+                a.out[m.unit * kPD + j] = __fmaf_rn(c, dj, wj);
+            } else if (m.exists) {
+                a.out[m.unit * kPD + j] = 0.f;
+                if (j == 0 && m.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
+            }
+        }
+        __syncthreads();
+
+        // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
+        if (any) {
+            const float4* dp = reinterpret_cast<const float4*>(delta_s + ui * kPD + 8 * cg);
+            const float4 d0 = dp[0], d1 = dp[1];
+            const float2 dl[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                                  make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
+            float amax[kPR];
+#pragma unroll
+            for (int i = 0; i < kPR; ++i) {
+                const float b = __fmul_rn(meta.beta, kval(i));
+#pragma unroll
+                for (int c = 0; c < 4; ++c) x[i][c] = __ffma2_rn(f2(b), dl[c], x[i][c]);
+                // row maxima of both units with full-warp reductions (the other
+                // half contributes 0, the smallest |x|)
+                const uint32_t mb = __float_as_uint(absmax8(x[i]));
+                const uint32_t m0 = __reduce_max_sync(0xffffffffu, ui ? 0u : mb);
+                const uint32_t m1 = __reduce_max_sync(0xffffffffu, ui ? mb : 0u);
+                amax[i] = __uint_as_float(ui ? m1 : m0);
+            }
+            if (cg == 0) {
+                reinterpret_cast<float4*>(rowbuf)[0] = make_float4(amax[0], amax[1], amax[2], amax[3]);
+                reinterpret_cast<float4*>(rowbuf)[1] = make_float4(amax[4], amax[5], amax[6], amax[7]);
+            }
+            __syncwarp();
+            if (cg < kPR) {
+                const uint32_t e = sdir[cg];
+                if (!(e >> 31)) {
+                    float scale, inv;
+                    row_scale(rowbuf[cg], scale, inv);
+                    rowbuf[kPR + cg] = inv;
+                    *reinterpret_cast<float*>(blk + ((e >> 16) & 0x7fffu)) = scale;
+                }
+            }
+            __syncwarp();
+            const float4 i0 = reinterpret_cast<const float4*>(rowbuf)[2];
+            const float4 i1 = reinterpret_cast<const float4*>(rowbuf)[3];
+            const float inv[kPR] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+            {
+                const uint4 d0 = reinterpret_cast<const uint4*>(sdir)[0];
+                const uint4 d1 = reinterpret_cast<const uint4*>(sdir)[1];
+                dir[0] = d0.x; dir[1] = d0.y; dir[2] = d0.z; dir[3] = d0.w;
+                dir[4] = d1.x; dir[5] = d1.y; dir[6] = d1.z; dir[7] = d1.w;
+            }
+#pragma unroll
+            for (int i = 0; i < kPR; ++i) {
+                const uint32_t e = dir[i], off = e & 0xffffu;
+                if (e >> 31) {
+                    const uint2 h0 = quant_fp16x4(x[i][0], x[i][1]);
+                    const uint2 h1 = quant_fp16x4(x[i][2], x[i][3]);
+                    *reinterpret_cast<uint4*>(const_cast<uint8_t*>(b16) + off) =
+                        make_uint4(h0.x, h0.y, h1.x, h1.y);
+                } else {
+                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + off) =
+                        make_uint2(quant_int8x4(x[i][0], x[i][1], inv[i]),
+                                   quant_int8x4(x[i][2], x[i][3], inv[i]));
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        __syncthreads();
+
+        // ---- write back (one bulk store per block)
+        if (tid == 0) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+                const PMeta m = *reinterpret_cast<const PMeta*>(st + a.st_meta + w * sizeof(PMeta));
+                if (m.active == 1)
+                    bulk_s2g(a.blocks + m.boff, smem_u32(st + w * a.block_stride), a.block_stride);
+            }
+            bulk_commit();
+        }
+        if (++stage == NS) {
+            stage = 0;
+            parity ^= 1u;
+        }
+    }
+
+    if (tid == 0) {
+        if (aborted) {
+            atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
+            for (int j = 0; j <= ahead; ++j) {
+                const int jt = it + j;
+                if (jt >= my_items) break;
+                (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
+                                        100000000ull);
+            }
+        }
+        bulk_wait_all<0>();
+    }
+}
+
+// Stage layout of the pair kernel; returns the number of stages that fit
+// (0 when fewer than three do).
+uint32_t pair_layout(StepArgs& a, bool kda, bool bf16) {
+    const uint32_t elt = bf16 ? 2 : 4;
+    auto up = [](uint32_t x, uint32_t m) { return (x + m - 1) / m * m; };
+    uint32_t off = 2 * a.block_stride;
+    a.st_q = off;
+    off = up(off + 2 * kPD * elt, 16);
+    a.st_k = off;
+    off = up(off + 2 * kPD * elt, 16);
+    a.st_v = off;
+    off = up(off + 2 * kPD * elt, 16);
+    a.st_alpha = off;
+    off += kda ? 2 * kPD * 4 : 0;
+    a.st_mask = off;
+    a.st_dir = off;
+    off += kPD * 4;
+    a.st_meta = off;
+    off += 2 * sizeof(PMeta);
+    a.stage_bytes = up(off, 128);
+    const uint32_t scratch = up((2 * 2 * kPG * kPD + 2 * kPD + 2 * kPG + kPG * 2 * 16) * 4, 128);
+    const uint32_t budget = 227u * 1024u;
+    uint32_t ns = (budget - scratch - 128) / a.stage_bytes;
+    if (ns > 6) ns = 6;
+    if (ns < 3) return 0;
+    a.n_stages = (int)ns;
+    a.scratch_off = ns * a.stage_bytes;
+    a.bar_off = a.scratch_off + scratch;
+    return ns;
+}
+
+template <bool KDA, bool BF16>
+cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    auto kern = decode_pair_kernel<KDA, BF16>;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        227 * 1024);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    StepArgs a = a0;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const uint32_t ns = pair_layout(a, KDA, BF16);
+    if (ns == 0) return cudaErrorInvalidConfiguration;
+    const size_t smem = a.bar_off + 8u * ns;
+    const int grid = std::min(a.n_items, sms);
+    kern<<<grid, kPT, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate) {
+    StepArgs b = a;
+    return pair_layout(b, gate == DAMP_GATE_VECTOR, in_dtype == DAMP_DTYPE_BF16) != 0;
+}
+
+cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, cudaStream_t stream) {
+    const bool kda = gate == DAMP_GATE_VECTOR, bf = in_dtype == DAMP_DTYPE_BF16;
+    if (kda) return bf ? launch_pair_t<true, true>(a, stream) : launch_pair_t<true, false>(a, stream);
+    return bf ? launch_pair_t<false, true>(a, stream) : launch_pair_t<false, false>(a, stream);
+}
+
+}  // namespace damp

@@ -71,6 +71,10 @@ struct CodecArgs {
 // Launchers (damp_decode.cu, damp_codec.cu).  They return cudaError_t.
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream);
+// d = 128 quantized states, two units of one head per CTA iteration
+// (damp_decode_pair.cu); a.n_items counts pairs x heads.
+cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, cudaStream_t stream);
+bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate);   // >= 3 stages fit
 cudaError_t launch_pack(const PoolDesc& p, const CodecArgs& a, cudaStream_t stream);
 cudaError_t launch_unpack(const PoolDesc& p, const CodecArgs& a, cudaStream_t stream);
 
