@@ -52,8 +52,15 @@ def lib():
                                           ctypes.c_float, P, P]
         _lib.oracle_decode_step.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P,
                                             P, P, P, P, P, P]
+        _lib.oracle_row_quant_error.restype = ctypes.c_double
+        _lib.oracle_row_quant_error.argtypes = [P, I]
+        _lib.oracle_calib_accumulate.argtypes = [I, I, I, I, I, I, P, P, P, P]
+        _lib.oracle_calib_scores.argtypes = [I, I, P, P]
+        _lib.oracle_calib_select.argtypes = [I, I, I, P, P]
+        _lib.oracle_calib_select_budget.argtypes = [I, I, I, P, P, P]
         for f in ("oracle_pack_unit", "oracle_unpack_unit", "oracle_step_unit",
-                  "oracle_decode_step"):
+                  "oracle_decode_step", "oracle_calib_accumulate", "oracle_calib_scores",
+                  "oracle_calib_select", "oracle_calib_select_budget"):
             getattr(_lib, f).restype = I
     return _lib
 
@@ -211,3 +218,60 @@ def decode_step(pool: State, gate: int, is_fp16, slot_idx, q, k, v, alpha, beta)
         raise ValueError("slot index out of range")
     assert rc == 0, rc
     return o
+
+
+# --------------------------------------------------------------------------
+# offline calibration (calib_oracle.c)
+# --------------------------------------------------------------------------
+
+def row_quant_error(x) -> float:
+    """Squared error of the INT8 row quantizer on one row (double)."""
+    x = _c(x, np.float32)
+    return float(lib().oracle_row_quant_error(_p(x), x.size))
+
+
+def calib_acc(H: int, dk: int) -> np.ndarray:
+    """Zeroed accumulator: energy [H][d_k], retention [H][d_k], count [H]."""
+    return np.zeros(2 * H * dk + H, np.float64)
+
+
+def calib_accumulate(acc: np.ndarray, gate: int, f32_pool, slot_idx, alpha) -> None:
+    """Add one step's records (FP32 states after the step) to ``acc``."""
+    f32_pool = _c(f32_pool, np.float32)
+    n_slots, H, dk, dv = f32_pool.shape
+    slot_idx = _c(slot_idx, np.int32)
+    alpha = _c(alpha, np.float32)
+    assert acc.dtype == np.float64 and acc.size == 2 * H * dk + H
+    rc = lib().oracle_calib_accumulate(gate, slot_idx.size, H, dk, dv, n_slots, _p(f32_pool),
+                                       _p(slot_idx), _p(alpha), _p(acc))
+    if rc == -2:
+        raise ValueError("slot index out of range")
+    assert rc == 0, rc
+
+
+def calib_scores(acc: np.ndarray, H: int, dk: int) -> np.ndarray:
+    score = np.empty((H, dk), np.float64)
+    rc = lib().oracle_calib_scores(H, dk, _p(_c(acc, np.float64)), _p(score))
+    assert rc == 0, rc
+    return score
+
+
+def calib_select(score, hp: int) -> np.ndarray:
+    """hp_row_idx uint16 [H][hp], ascending per head."""
+    score = _c(score, np.float64)
+    H, dk = score.shape
+    out = np.zeros((H, hp), np.uint16)
+    rc = lib().oracle_calib_select(H, dk, hp, _p(score), _p(out))
+    assert rc == 0, rc
+    return out
+
+
+def calib_select_budget(score, budget: int):
+    """(is_fp16 uint8 [H][d_k], hp int32 [H]) for a total of ``budget`` FP16 rows."""
+    score = _c(score, np.float64)
+    H, dk = score.shape
+    is16 = np.zeros((H, dk), np.uint8)
+    hp = np.zeros(H, np.int32)
+    rc = lib().oracle_calib_select_budget(H, dk, budget, _p(score), _p(is16), _p(hp))
+    assert rc == 0, rc
+    return is16, hp

@@ -9,7 +9,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "damp_oracle.c")
+SRCS = [os.path.join(HERE, f) for f in ("damp_oracle.c", "calib_oracle.c")]
 LIB = os.path.join(HERE, "liboracle.so")
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
@@ -17,9 +17,10 @@ CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-s
 
 
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+    if not force and os.path.exists(LIB) and \
+            all(os.path.getmtime(LIB) >= os.path.getmtime(s) for s in SRCS):
         return LIB
-    cmd = ["gcc", *CFLAGS, "-o", LIB, SRC, "-lm"]
+    cmd = ["gcc", *CFLAGS, "-o", LIB, *SRCS, "-lm"]
     subprocess.run(cmd, check=True)
     return LIB
 
