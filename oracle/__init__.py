@@ -9,7 +9,8 @@ the CUDA library and never imports it.
 Logical state of a quantized (slot, head) state, rows in key-channel order:
 ``scale`` float32 [..., d_k], ``half`` uint16 [..., d_k, d_v] (binary16 bits of
 FP16 rows), ``code`` int8 [..., d_k, d_v] (codes of INT8 rows); unused entries
-are zero.  An FP32 state is ``f32`` float32 [..., d_k, d_v].
+are zero.  The FP8 comparison format uses ``scale`` and ``code`` (E4M3 bit
+patterns, viewed as int8) for every row.  An FP32 state is ``f32`` float32 [..., d_k, d_v].
 """
 from __future__ import annotations
 
@@ -23,6 +24,7 @@ from . import build as _build
 
 FMT_FP32 = 0
 FMT_QUANT = 1
+FMT_FP8 = 2
 GATE_SCALAR = 0
 GATE_VECTOR = 1
 
@@ -43,6 +45,9 @@ def lib():
         _lib.oracle_f16_from_f32_array.argtypes = [P, P, ctypes.c_long]
         _lib.oracle_f32_from_f16_array.argtypes = [P, P, ctypes.c_long]
         _lib.oracle_quantize_row.argtypes = [P, I, P, P]
+        _lib.oracle_quantize_row_fp8.argtypes = [P, I, P, P]
+        _lib.oracle_e4m3_from_f32_array.argtypes = [P, P, ctypes.c_long]
+        _lib.oracle_f32_from_e4m3_array.argtypes = [P, P, ctypes.c_long]
         _lib.oracle_quantize_row_prerounding.argtypes = [P, I, P]
         _lib.oracle_pairwise_sum.restype = ctypes.c_float
         _lib.oracle_pairwise_sum.argtypes = [P, I]
@@ -97,6 +102,30 @@ def quantize_row(x):
     code = np.empty(x.shape, np.int8)
     scale = np.zeros(1, np.float32)
     lib().oracle_quantize_row(_p(x), x.size, _p(code), _p(scale))
+    return code, scale[0]
+
+
+def e4m3_from_f32(x) -> np.ndarray:
+    """E4M3 codes (uint8 bit patterns), nearest-even with saturation at 448."""
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().oracle_e4m3_from_f32_array(_p(x), _p(out), x.size)
+    return out
+
+
+def f32_from_e4m3(c) -> np.ndarray:
+    c = _c(c, np.uint8)
+    out = np.empty(c.shape, np.float32)
+    lib().oracle_f32_from_e4m3_array(_p(c), _p(out), c.size)
+    return out
+
+
+def quantize_row_fp8(x):
+    """(E4M3 codes uint8[n], scale float32) of one FP8 row."""
+    x = _c(x, np.float32)
+    code = np.empty(x.shape, np.uint8)
+    scale = np.zeros(1, np.float32)
+    lib().oracle_quantize_row_fp8(_p(x), x.size, _p(code), _p(scale))
     return code, scale[0]
 
 

@@ -42,6 +42,18 @@
  *      FP32 state X read out exactly, up to double rounding).
  *   R8 FP16 rows are rounded to nearest, ties to even, with IEEE overflow to
  *      infinity; subnormals are kept.
+ *
+ * FP8 comparison format ([DAMP-v1] names uniform FP8 as a baseline that
+ * already loses accuracy; it does not fix the variant or the scaling):
+ *   F1 every row is FP8 E4M3 as defined by the OCP 8-bit floating point
+ *      specification: sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ *      subnormals, no infinities, S.1111.111 is NaN, largest finite 448.
+ *   F2 per-row absmax scaling as for INT8 rows: scale = fl(a/448),
+ *      inv = fl(448/a); a == 0 or inv == +inf -> scale 0, codes 0.
+ *   F3 code = the E4M3 value nearest to the FP32 product fl(x*inv), ties to
+ *      the even mantissa; magnitudes above 448 saturate to 448.  (The
+ *      product is rounded to FP32 first, as a conversion from FP32 does.)
+ *   F4 dequantize: fl(value(code) * scale).
  */
 #include <math.h>
 #include <stddef.h>
@@ -51,6 +63,7 @@
 
 #define ORACLE_FMT_FP32 0   /* plain FP32 state, no quantization            */
 #define ORACLE_FMT_QUANT 1  /* FP16 rows where is_fp16[i], INT8 rows elsewhere */
+#define ORACLE_FMT_FP8 2    /* every row FP8 E4M3 with an FP32 scale (F1-F4)   */
 
 #define ORACLE_GATE_SCALAR 0 /* GDN: one decay per (slot, head)             */
 #define ORACLE_GATE_VECTOR 1 /* KDA: one decay per key channel               */
@@ -157,6 +170,73 @@ void oracle_quantize_row_prerounding(const float* x, int n, double* t_out)
 }
 
 /* ------------------------------------------------------------------------ */
+/* FP8 E4M3 (F1-F4)                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Value of an E4M3 code (F1). */
+float oracle_f32_from_e4m3(uint8_t c)
+{
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);             /* subnormal: m * 2^-6 / 8 */
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return (float)(sign ? -v : v);
+}
+
+/* Nearest E4M3 code to y, ties to even mantissa, saturating at 448 (F3).
+ * The magnitude is scaled (exactly, by a power of two) to units of the E4M3
+ * quantum at its exponent and rounded with nearbyint(). */
+uint8_t oracle_e4m3_from_f32(float y)
+{
+    uint8_t sign = signbit(y) ? 0x80u : 0u;
+    if (isnan(y)) return (uint8_t)(sign | 0x7fu);
+    double a = fabs((double)y);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7eu);
+    if (a < ldexp(1.0, -6)) {
+        double m = nearbyint(ldexp(a, 9));            /* quantum 2^-9 */
+        return (uint8_t)(sign | (uint8_t)m);          /* m == 8 is the smallest normal */
+    }
+    int e;
+    frexp(a, &e);                                     /* a = f * 2^e, f in [0.5, 1) */
+    int E = e - 1;                                    /* a in [2^E, 2^(E+1)) */
+    double r = nearbyint(ldexp(a, 3 - E));            /* in [8, 16] */
+    if (r == 16.0) {
+        r = 8.0;
+        E += 1;
+    }
+    return (uint8_t)(sign | (uint8_t)((E + 7) << 3) | (uint8_t)(r - 8.0));
+}
+
+void oracle_e4m3_from_f32_array(const float* x, uint8_t* out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = oracle_e4m3_from_f32(x[i]);
+}
+
+void oracle_f32_from_e4m3_array(const uint8_t* c, float* out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = oracle_f32_from_e4m3(c[i]);
+}
+
+/* F2, F3 for one row; codes are stored as the E4M3 bit patterns. */
+void oracle_quantize_row_fp8(const float* x, int n, uint8_t* code, float* scale)
+{
+    float amax = 0.0f;
+    for (int j = 0; j < n; ++j) {
+        float t = fabsf(x[j]);
+        if (t > amax) amax = t;
+    }
+    float inv = 448.0f / amax;
+    if (amax == 0.0f || isinf(inv)) {
+        *scale = 0.0f;
+        for (int j = 0; j < n; ++j) code[j] = 0;
+        return;
+    }
+    *scale = amax / 448.0f;
+    for (int j = 0; j < n; ++j) code[j] = oracle_e4m3_from_f32(x[j] * inv);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Pairwise FP32 sum (R5)                                                    */
 /* ------------------------------------------------------------------------ */
 
@@ -189,6 +269,14 @@ int oracle_pack_unit(int fmt, int dk, int dv, const uint8_t* is_fp16, const floa
         memcpy(f32, S, sizeof(float) * (size_t)dk * (size_t)dv);
         return ORACLE_OK;
     }
+    if (fmt == ORACLE_FMT_FP8) {
+        for (int i = 0; i < dk; ++i) {
+            oracle_quantize_row_fp8(S + (size_t)i * dv, dv, (uint8_t*)code + (size_t)i * dv,
+                                    &scale[i]);
+            for (int j = 0; j < dv; ++j) half[(size_t)i * dv + j] = 0;
+        }
+        return ORACLE_OK;
+    }
     if (fmt != ORACLE_FMT_QUANT) return ORACLE_EINVAL;
     for (int i = 0; i < dk; ++i) {
         const float* row = S + (size_t)i * dv;
@@ -215,6 +303,14 @@ int oracle_unpack_unit(int fmt, int dk, int dv, const uint8_t* is_fp16, const fl
         memcpy(S, f32, sizeof(float) * (size_t)dk * (size_t)dv);
         return ORACLE_OK;
     }
+    if (fmt == ORACLE_FMT_FP8) {
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) {
+                size_t e = (size_t)i * dv + j;
+                S[e] = oracle_f32_from_e4m3((uint8_t)code[e]) * scale[i];
+            }
+        return ORACLE_OK;
+    }
     if (fmt != ORACLE_FMT_QUANT) return ORACLE_EINVAL;
     for (int i = 0; i < dk; ++i)
         for (int j = 0; j < dv; ++j) {
@@ -238,7 +334,8 @@ int oracle_step_unit(int fmt, int gate, int dk, int dv, const uint8_t* is_fp16,
                      const float* alpha, float beta, double* o, float* X_out)
 {
     if (dk <= 0 || dv <= 0) return ORACLE_EINVAL;
-    if (fmt != ORACLE_FMT_FP32 && fmt != ORACLE_FMT_QUANT) return ORACLE_EINVAL;
+    if (fmt != ORACLE_FMT_FP32 && fmt != ORACLE_FMT_QUANT && fmt != ORACLE_FMT_FP8)
+        return ORACLE_EINVAL;
     if (gate != ORACLE_GATE_SCALAR && gate != ORACLE_GATE_VECTOR) return ORACLE_EINVAL;
     size_t ne = (size_t)dk * dv;
     float* Shat = malloc(sizeof(float) * ne);
@@ -280,7 +377,8 @@ int oracle_step_unit(int fmt, int gate, int dk, int dv, const uint8_t* is_fp16,
     }
     if (X_out) memcpy(X_out, X, sizeof(float) * ne);
 
-    /* [STEP-C2] step 6 / [DAMP-v2]: requantize in place (FP16 rows, INT8 rows) */
+    /* [STEP-C2] step 6 / [DAMP-v2]: requantize in place (FP16 rows, INT8 rows;
+     * FP8 rows for the comparison format) */
     oracle_pack_unit(fmt, dk, dv, is_fp16, X, scale, half, code, f32);
 
     free(Shat); free(Sp); free(X); free(prod); free(delta); free(b);
