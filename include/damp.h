@@ -30,6 +30,12 @@
  *   INT8 rows: a = max_j |X_ij|; scale = fl(a/127); inv = fl(127/a);
  *              code = nearest integer to the exact X*inv, ties to even.
  *              a == 0 or inv == +inf -> scale 0, codes 0.
+ *   FP8 rows (DAMP_FMT_FP8_ROW, the uniform FP8 baseline the DAMP v1 abstract
+ *              names): E4M3 codes as the OCP 8-bit floating point
+ *              specification defines them; scale = fl(a/448); inv =
+ *              fl(448/a); code = the E4M3 value nearest to the FP32 product
+ *              fl(X*inv), ties to even, saturating at 448; dequantized as
+ *              fl(value * scale).  Same zero-row rule as INT8 rows.
  *
  * Conventions for every call:
  *   - Device memory is owned by the caller (for example allocated by
@@ -75,6 +81,7 @@ extern "C" {
 #define DAMP_FMT_FP32 0     /* plain FP32 state (the pages' unquantized baseline)   */
 #define DAMP_FMT_INT8_ROW 1 /* every row INT8 + FP32 absmax scale (uniform INT8)   */
 #define DAMP_FMT_MIXED 2    /* hp_rows FP16 key rows per head, the rest INT8 (DAMP) */
+#define DAMP_FMT_FP8_ROW 3  /* every row FP8 E4M3 + FP32 absmax scale (uniform FP8) */
 
 #define DAMP_GATE_SCALAR 0 /* GDN: alpha is one FP32 per (entry, head)            */
 #define DAMP_GATE_VECTOR 1 /* KDA: alpha is d_k FP32 per (entry, head)            */
@@ -99,6 +106,7 @@ const char* damp_status_string(int status);
  * Quantized block byte order: r FP32 scales (INT8 rows in increasing key
  * index) padded to 16 B, then the hp FP16 rows in increasing key index, then
  * the r INT8 rows in increasing key index.  FP32 blocks: row-major [d_k][d_v].
+ * FP8 blocks have the INT8-row layout with E4M3 bytes in place of INT8 codes.
  * Either output pointer may be NULL.
  */
 int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
@@ -106,8 +114,9 @@ int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
 
 /*
  * Bytes the caller must allocate for a pool of n_slots x H blocks: a header
- * (per-head FP16-row masks and the device status word, 256 B aligned)
- * followed by the blocks, block (slot, h) at header + (slot*H + h)*stride.
+ * (device status word, per-head FP16-row masks, row directory and block
+ * table, 256 B aligned) followed by the slots.  With one FP16-row count for
+ * every head, block (slot, h) is at header + (slot*H + h)*stride.
  */
 int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
                     size_t* bytes);
@@ -127,6 +136,27 @@ int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_row
 int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
                      const uint16_t* hp_row_idx, void* dev_buf, size_t buf_bytes,
                      damp_pool** out);
+
+/*
+ * Mixed pool whose heads hold different numbers of FP16 rows: the "fixed
+ * storage budget" of the DAMP later abstract (mlsanity.com index page) spent
+ * unevenly, e.g. as damp_calib_select_budget picks it.
+ *   is_fp16 : host array [H][d_k] of 0/1 bytes, 1 = FP16 key row.  Copied.
+ * Head h's block has the layout of damp_layout(DAMP_FMT_MIXED, d_k, d_v,
+ * hp_h) with hp_h the head's FP16-row count; a slot holds the H blocks one
+ * after another (damp_pool_head_layout gives each head's offset and size).
+ * Every other call treats such a pool like any DAMP_FMT_MIXED pool; a map
+ * with the same count in every head gives the pool damp_pool_create makes.
+ */
+int damp_pool_bytes_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is_fp16,
+                        size_t* bytes);
+int damp_pool_create_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is_fp16,
+                         void* dev_buf, size_t buf_bytes, damp_pool** out);
+
+/* Head h's block: algorithmic size, stride and byte offset inside a slot.
+ * Any output pointer may be NULL. */
+int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,
+                          size_t* block_stride, size_t* offset_in_slot);
 
 /* Release the descriptor (never the caller's device buffer).  NULL is a no-op. */
 int damp_pool_destroy(damp_pool* pool);
@@ -191,6 +221,62 @@ int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float
 int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
                             const uint16_t* half, const int8_t* code, const float* f32,
                             void* block);
+
+/* ---- offline calibration of the FP16 key rows ------------------------------
+ *
+ * Picks, per head, the key rows to keep in FP16 from a calibration run of the
+ * unquantized recurrence.  The pages ("DAMP: Decay-Aware Mixed-Precision
+ * Recurrent-State Quantization", both abstracts) select high-risk key channels
+ * offline from two signals, quantization-error energy and decay-based error
+ * retention, under a fixed storage budget; they give no formula.  Readings:
+ *   energy_i    += sum_j (X_ij - fl(c_ij * s_i))^2     (double)
+ *                  for the FP32 state X after a step, with c, s the decode
+ *                  step's own INT8 quantizer applied to row i;
+ *   retention_i += alpha_i^2                           (double; GDN: the
+ *                  scalar decay of the (entry, head), KDA: channel i);
+ *   count       += 1 per recorded (entry, head);
+ *   score_i      = (energy_i / count) / max(1 - retention_i / count, 2^-30)
+ *                  (error injected every step and multiplied by alpha_i^2 per
+ *                  step accumulates as a geometric series).
+ * Selection: per head the hp_rows largest scores (ties: lower row), or the
+ * `budget` largest over all heads (ties: lower head, then lower row).
+ *
+ * Accumulator: caller-owned device memory of damp_calib_bytes(H, d_k) bytes,
+ * 8-byte aligned, zeroed by the caller before the first accumulate; layout
+ * double energy[H][d_k], retention[H][d_k], count[H].  Accumulation is
+ * deterministic: each (head, row) total is owned by one warp that adds the
+ * batch entries in order.
+ */
+size_t damp_calib_bytes(int H, int d_k);
+
+/*
+ * Add one step's records.  `pool` must be a DAMP_FMT_FP32 pool holding the
+ * states after the step (for example right after damp_decode_step on it);
+ * slot_idx [n] (device int32) names the entries stepped, negative entries are
+ * skipped, entries >= n_slots set DAMP_EFLAG_SLOT_RANGE and are skipped;
+ * alpha is the step's decay, [n][H] (gate DAMP_GATE_SCALAR) or [n][H][d_k]
+ * (DAMP_GATE_VECTOR) FP32 on the device.
+ */
+int damp_calib_accumulate(const damp_pool* pool, int n, const int32_t* slot_idx, int gate,
+                          const float* alpha, double* acc, void* stream);
+
+/*
+ * Scores and per-head selection.  score [H][d_k] (device double, may be NULL)
+ * receives every score; hp_row_idx [H][hp_rows] (device uint16) receives the
+ * selected rows of each head in increasing order, ready for
+ * damp_pool_create.  0 <= hp_rows <= d_k.
+ */
+int damp_calib_select(int H, int d_k, int hp_rows, const double* acc, double* score,
+                      uint16_t* hp_row_idx, void* stream);
+
+/*
+ * Selection under one budget shared by the H heads: is_fp16 [H][d_k] (device
+ * uint8, 1 = FP16 row) and hp_per_head [H] (device int32).  score [H][d_k]
+ * (device double) is required here: it holds the scores the ranking reads.
+ * 0 <= budget <= H*d_k.
+ */
+int damp_calib_select_budget(int H, int d_k, int budget, const double* acc, double* score,
+                             uint8_t* is_fp16, int32_t* hp_per_head, void* stream);
 
 #ifdef __cplusplus
 }

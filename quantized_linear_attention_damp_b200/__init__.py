@@ -33,12 +33,14 @@ DAMP_EFLAG_TIMEOUT = 2
 DAMP_FMT_FP32 = 0
 DAMP_FMT_INT8_ROW = 1
 DAMP_FMT_MIXED = 2
+DAMP_FMT_FP8_ROW = 3
 DAMP_GATE_SCALAR = 0
 DAMP_GATE_VECTOR = 1
 DAMP_DTYPE_BF16 = 0
 DAMP_DTYPE_F32 = 1
 
-FORMATS = {"fp32": DAMP_FMT_FP32, "int8": DAMP_FMT_INT8_ROW, "mixed": DAMP_FMT_MIXED}
+FORMATS = {"fp32": DAMP_FMT_FP32, "int8": DAMP_FMT_INT8_ROW, "mixed": DAMP_FMT_MIXED,
+           "fp8": DAMP_FMT_FP8_ROW}
 
 
 class DampError(RuntimeError):
@@ -67,6 +69,14 @@ def _load():
         "damp_pool_get_error": (I, [P, ctypes.POINTER(ctypes.c_uint32), I, P]),
         "damp_block_to_logical": (I, [P, I, P, P, P, P, P]),
         "damp_block_from_logical": (I, [P, I, P, P, P, P, P]),
+        "damp_pool_bytes_map": (I, [I, I, I, I, P, ctypes.POINTER(S)]),
+        "damp_pool_create_map": (I, [I, I, I, I, P, P, S, ctypes.POINTER(P)]),
+        "damp_pool_head_layout": (I, [P, I, ctypes.POINTER(S), ctypes.POINTER(S),
+                                      ctypes.POINTER(S)]),
+        "damp_calib_bytes": (S, [I, I]),
+        "damp_calib_accumulate": (I, [P, I, P, I, P, P, P]),
+        "damp_calib_select": (I, [I, I, I, P, P, P, P]),
+        "damp_calib_select_budget": (I, [I, I, I, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -150,6 +160,39 @@ def damp_pool_create(format: int, n_slots: int, H: int, d_k: int, d_v: int, hp_r
     _check(_lib.damp_pool_create(format, n_slots, H, d_k, d_v, hp_rows, _ptr(idx), buf_ptr,
                                  nbytes, ctypes.byref(h)), "damp_pool_create")
     return h.value
+
+
+def damp_pool_bytes_map(n_slots: int, H: int, d_k: int, d_v: int, is_fp16) -> int:
+    m = np.ascontiguousarray(is_fp16, np.uint8)
+    if m.shape != (H, d_k):
+        raise ValueError("is_fp16 must be [H][d_k]")
+    out = ctypes.c_size_t()
+    _check(_lib.damp_pool_bytes_map(n_slots, H, d_k, d_v, _ptr(m), ctypes.byref(out)),
+           "damp_pool_bytes_map")
+    return out.value
+
+
+def damp_pool_create_map(n_slots: int, H: int, d_k: int, d_v: int, is_fp16, buf) -> int:
+    """Mixed pool with a per-head FP16-row map (counts may differ per head)."""
+    m = np.ascontiguousarray(is_fp16, np.uint8)
+    if m.shape != (H, d_k):
+        raise ValueError("is_fp16 must be [H][d_k]")
+    h = ctypes.c_void_p()
+    ptr, nbytes = None, 0
+    if buf is not None:
+        _cuda(buf, torch.uint8, "dev_buf")
+        ptr, nbytes = _ptr(buf), buf.numel()
+    _check(_lib.damp_pool_create_map(n_slots, H, d_k, d_v, _ptr(m), ptr, nbytes,
+                                     ctypes.byref(h)), "damp_pool_create_map")
+    return h.value
+
+
+def damp_pool_head_layout(pool: int, h: int) -> tuple[int, int, int]:
+    """(block_bytes, block_stride, offset_in_slot) of head h."""
+    b, s, o = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.damp_pool_head_layout(pool, h, ctypes.byref(b), ctypes.byref(s),
+                                      ctypes.byref(o)), "damp_pool_head_layout")
+    return b.value, s.value, o.value
 
 
 def damp_pool_destroy(pool: int) -> None:
@@ -237,22 +280,95 @@ def damp_pool_get_error(pool: int, clear: bool = False, stream=None, device=None
     return f.value
 
 
+# ---------------------------------------------------------------- calibration
+
+def damp_calib_bytes(H: int, d_k: int) -> int:
+    return int(_lib.damp_calib_bytes(H, d_k))
+
+
+def calib_acc(H: int, d_k: int, device="cuda") -> torch.Tensor:
+    """Zeroed calibration accumulator (float64): energy [H][d_k], retention
+    [H][d_k], count [H]."""
+    return torch.zeros(damp_calib_bytes(H, d_k) // 8, dtype=torch.float64, device=device)
+
+
+def damp_calib_accumulate(pool: int, slot_idx: torch.Tensor, alpha: torch.Tensor,
+                          acc: torch.Tensor, stream=None) -> None:
+    """Add one step's records of an FP32 pool (states after the step)."""
+    _cuda(slot_idx, torch.int32, "slot_idx")
+    _cuda(alpha, torch.float32, "alpha")
+    _cuda(acc, torch.float64, "acc")
+    gate = DAMP_GATE_VECTOR if alpha.dim() == 3 else DAMP_GATE_SCALAR
+    _check(_lib.damp_calib_accumulate(pool, slot_idx.numel(), _ptr(slot_idx), gate, _ptr(alpha),
+                                      _ptr(acc), _stream(stream, acc.device)),
+           "damp_calib_accumulate")
+
+
+def damp_calib_select(H: int, d_k: int, hp_rows: int, acc: torch.Tensor, score=None,
+                      hp_row_idx=None, stream=None):
+    """Per-head selection; returns (hp_row_idx [H][hp_rows], score float64
+    [H][d_k]).  Row indices are int16 (every index is below d_k <= 128)."""
+    _cuda(acc, torch.float64, "acc")
+    if score is None:
+        score = torch.empty((H, d_k), dtype=torch.float64, device=acc.device)
+    if hp_row_idx is None:
+        hp_row_idx = torch.empty((H, hp_rows), dtype=torch.int16, device=acc.device)
+    _cuda(score, torch.float64, "score")
+    _cuda(hp_row_idx, torch.int16, "hp_row_idx")
+    _check(_lib.damp_calib_select(H, d_k, hp_rows, _ptr(acc), _ptr(score), _ptr(hp_row_idx),
+                                  _stream(stream, acc.device)), "damp_calib_select")
+    return hp_row_idx, score
+
+
+def damp_calib_select_budget(H: int, d_k: int, budget: int, acc: torch.Tensor, stream=None):
+    """Selection under a budget shared by all heads; returns (is_fp16 uint8
+    [H][d_k], hp_per_head int32 [H], score float64 [H][d_k])."""
+    _cuda(acc, torch.float64, "acc")
+    score = torch.empty((H, d_k), dtype=torch.float64, device=acc.device)
+    is16 = torch.empty((H, d_k), dtype=torch.uint8, device=acc.device)
+    hp = torch.empty(H, dtype=torch.int32, device=acc.device)
+    _check(_lib.damp_calib_select_budget(H, d_k, budget, _ptr(acc), _ptr(score), _ptr(is16),
+                                         _ptr(hp), _stream(stream, acc.device)),
+           "damp_calib_select_budget")
+    return is16, hp, score
+
+
 # ---------------------------------------------------------------- convenience
 
 class DampPool:
-    """A pool buffer (allocated by PyTorch) bound to a libdamp descriptor."""
+    """A pool buffer (allocated by PyTorch) bound to a libdamp descriptor.
+
+    ``hp_row_idx`` [H][hp] gives every head the same FP16-row count;
+    ``fp16_map`` [H][d] (0/1, mixed format only) lets the count differ per
+    head."""
 
     def __init__(self, fmt, n_slots: int, H: int, d: int, hp_row_idx=None,
-                 device="cuda"):
+                 device="cuda", fp16_map=None):
         self.fmt = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
-        hp_row_idx = None if hp_row_idx is None else np.asarray(hp_row_idx).reshape(H, -1)
-        self.hp = 0 if hp_row_idx is None else hp_row_idx.shape[1]
         self.n_slots, self.H, self.d = n_slots, H, d
-        self.block_bytes, self.block_stride = damp_layout(self.fmt, d, d, self.hp)
-        self.nbytes = damp_pool_bytes(self.fmt, n_slots, H, d, d, self.hp)
-        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
-        self.handle = damp_pool_create(self.fmt, n_slots, H, d, d, self.hp, hp_row_idx, self.buf)
+        if fp16_map is not None:
+            if self.fmt != DAMP_FMT_MIXED:
+                raise ValueError("an FP16-row map needs the mixed format")
+            fp16_map = np.ascontiguousarray(fp16_map, np.uint8).reshape(H, d)
+            self.nbytes = damp_pool_bytes_map(n_slots, H, d, d, fp16_map)
+            self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+            self.handle = damp_pool_create_map(n_slots, H, d, d, fp16_map, self.buf)
+            counts = fp16_map.sum(axis=1)
+            self.hp = int(counts[0]) if (counts == counts[0]).all() else -1
+        else:
+            hp_row_idx = None if hp_row_idx is None else np.asarray(hp_row_idx).reshape(H, -1)
+            self.hp = 0 if hp_row_idx is None else hp_row_idx.shape[1]
+            self.nbytes = damp_pool_bytes(self.fmt, n_slots, H, d, d, self.hp)
+            self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+            self.handle = damp_pool_create(self.fmt, n_slots, H, d, d, self.hp, hp_row_idx,
+                                           self.buf)
         self.header_bytes = damp_pool_block_offset(self.handle, 0, 0)
+        self.heads = [damp_pool_head_layout(self.handle, h) for h in range(H)]
+        self.slot_stride = sum(st for _, st, _ in self.heads)
+        strides = {st for _, st, _ in self.heads}
+        self.block_stride = max(strides)
+        self.block_bytes = max(b for b, _, _ in self.heads)
+        self.uniform = len(strides) == 1
 
     def close(self):
         if getattr(self, "handle", None):
@@ -265,9 +381,21 @@ class DampPool:
         except Exception:
             pass
 
+    def slots(self) -> torch.Tensor:
+        """View of the slot area: uint8 [n_slots][slot_stride]."""
+        return self.buf[self.header_bytes:].view(self.n_slots, self.slot_stride)
+
     def blocks(self) -> torch.Tensor:
-        """View of the block area: uint8 [n_slots][H][block_stride]."""
-        return self.buf[self.header_bytes:].view(self.n_slots, self.H, self.block_stride)
+        """View of the blocks: uint8 [n_slots][H][block_stride] (every head the
+        same block size)."""
+        if not self.uniform:
+            raise ValueError("heads differ in block size; use slots() / block()")
+        return self.slots().view(self.n_slots, self.H, self.block_stride)
+
+    def block(self, slot: int, h: int) -> torch.Tensor:
+        """View of block (slot, h): uint8 [head block stride]."""
+        _, st, off = self.heads[h]
+        return self.slots()[slot, off:off + st]
 
     def pack(self, slot_idx, state, stream=None):
         damp_pool_pack(self.handle, slot_idx, state, stream)
@@ -282,13 +410,14 @@ class DampPool:
         return damp_pool_get_error(self.handle, clear, stream, self.buf.device)
 
     def read_logical(self, slots=None) -> dict:
-        """Logical form of blocks [len(slots)][H] (host numpy), via one D2H copy."""
-        raw = self.blocks().cpu().numpy()
-        slots = range(self.n_slots) if slots is None else slots
+        """Logical form of blocks [len(slots)][H] (host numpy)."""
+        slots = list(range(self.n_slots)) if slots is None else [int(x) for x in slots]
+        raw = self.slots()[torch.as_tensor(slots, device=self.buf.device)].cpu().numpy()
         out = None
-        for i, s in enumerate(slots):
+        for i in range(len(slots)):
             for h in range(self.H):
-                lg = damp_block_to_logical(self.handle, h, raw[s, h], self.fmt, self.d)
+                _, st, off = self.heads[h]
+                lg = damp_block_to_logical(self.handle, h, raw[i, off:off + st], self.fmt, self.d)
                 if out is None:
                     out = {k: np.empty((len(slots), self.H) + v.shape, v.dtype)
                            for k, v in lg.items()}
@@ -298,7 +427,7 @@ class DampPool:
 
     def write_logical(self, slot: int, logical: dict):
         """Write the logical form [H][...] of one slot into the pool (host -> device)."""
-        raw = np.stack([damp_block_from_logical(self.handle, h, self.block_stride,
-                                                **{k: v[h] for k, v in logical.items()})
-                        for h in range(self.H)])
-        self.blocks()[slot].copy_(torch.from_numpy(raw))
+        raw = np.concatenate([damp_block_from_logical(self.handle, h, self.heads[h][1],
+                                                      **{k: v[h] for k, v in logical.items()})
+                              for h in range(self.H)])
+        self.slots()[slot].copy_(torch.from_numpy(raw))

@@ -26,7 +26,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(int format, int d_k, int d_v, int hp_rows) {
-    if (format != DAMP_FMT_FP32 && format != DAMP_FMT_INT8_ROW && format != DAMP_FMT_MIXED)
+    if (format != DAMP_FMT_FP32 && format != DAMP_FMT_INT8_ROW && format != DAMP_FMT_MIXED &&
+        format != DAMP_FMT_FP8_ROW)
         return DAMP_ERR_INVALID_ARGUMENT;
     if (hp_rows < 0 || hp_rows > d_k) return DAMP_ERR_INVALID_ARGUMENT;
     if (format != DAMP_FMT_MIXED && hp_rows != 0) return DAMP_ERR_INVALID_ARGUMENT;
@@ -52,7 +53,7 @@ void layout(int format, int d, int hp, size_t* bytes, size_t* stride, uint32_t* 
 }
 
 size_t header_bytes(int H) {
-    return align_up(damp::dir_offset(H) + (size_t)H * damp::kDirWords * 4, 256);
+    return align_up(damp::head_table_offset(H) + (size_t)H * 16, 256);
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? DAMP_OK : DAMP_ERR_CUDA; }
@@ -89,6 +90,44 @@ int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
     return DAMP_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Per-head layout of a pool whose FP16-row masks are known: the block table
+// (offset inside the slot, stride, FP16-row offset, INT8-row offset), the
+// slot stride, the largest block size and stride.
+struct Layout {
+    std::vector<uint32_t> heads;   // [H][4]
+    size_t slot_stride = 0, max_bytes = 0, max_stride = 0;
+};
+
+Layout pool_layout(int format, int H, int d, const std::vector<uint32_t>& masks) {
+    Layout L;
+    L.heads.assign((size_t)H * 4, 0u);
+    for (int h = 0; h < H; ++h) {
+        int hp = 0;
+        for (int w = 0; w < damp::kMaskWords; ++w)
+            hp += __builtin_popcount(masks[(size_t)h * damp::kMaskWords + w]);
+        size_t b, st;
+        uint32_t f16, i8;
+        layout(format, d, hp, &b, &st, &f16, &i8);
+        uint32_t* e = &L.heads[(size_t)h * 4];
+        e[0] = (uint32_t)L.slot_stride;
+        e[1] = (uint32_t)st;
+        e[2] = f16;
+        e[3] = i8;
+        L.slot_stride += st;
+        if (b > L.max_bytes) L.max_bytes = b;
+        if (st > L.max_stride) L.max_stride = st;
+    }
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
 int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
                     size_t* bytes) {
     if (!bytes || n_slots < 1 || H < 1) return DAMP_ERR_INVALID_ARGUMENT;
@@ -100,6 +139,100 @@ int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_row
     *bytes = header_bytes(H) + (size_t)n_slots * H * s;
     return DAMP_OK;
 }
+
+}  // extern "C"
+
+namespace {
+
+// Masks from a per-head FP16-row map (0/1 bytes, [H][d_k]).
+int masks_from_map(int H, int d_k, const uint8_t* is_fp16, std::vector<uint32_t>* masks) {
+    masks->assign((size_t)H * damp::kMaskWords, 0u);
+    for (int h = 0; h < H; ++h)
+        for (int i = 0; i < d_k; ++i) {
+            const uint8_t f = is_fp16[(size_t)h * d_k + i];
+            if (f > 1) return DAMP_ERR_INVALID_ARGUMENT;
+            if (f) (*masks)[(size_t)h * damp::kMaskWords + (i >> 5)] |= 1u << (i & 31);
+        }
+    return DAMP_OK;
+}
+
+int create_common(int format, int n_slots, int H, int d_k, int hp_rows,
+                  const std::vector<uint32_t>& masks, void* dev_buf, size_t buf_bytes,
+                  damp_pool** out) {
+    const Layout L = pool_layout(format, H, d_k, masks);
+    if (L.slot_stride > 0xffffffffull) return DAMP_ERR_UNSUPPORTED;
+    PoolDesc d{};
+    d.format = format;
+    d.n_slots = n_slots;
+    d.H = H;
+    d.d = d_k;
+    d.hp = hp_rows;
+    d.block_bytes = L.max_bytes;
+    d.block_stride = L.max_stride;
+    d.slot_stride = L.slot_stride;
+    d.header_bytes = header_bytes(H);
+    d.dir_off = damp::dir_offset(H);
+    d.head_off = damp::head_table_offset(H);
+    d.pool_bytes = d.header_bytes + (size_t)n_slots * d.slot_stride;
+    if (dev_buf) {
+        if (!aligned16(dev_buf)) return DAMP_ERR_MISALIGNED;
+        if (buf_bytes < d.pool_bytes) return DAMP_ERR_BUFFER_TOO_SMALL;
+    }
+    damp_pool* p = new (std::nothrow) damp_pool;
+    if (!p) return DAMP_ERR_INVALID_ARGUMENT;
+    p->d = d;
+    p->d.dev_buf = static_cast<uint8_t*>(dev_buf);
+    p->d.host_masks = new (std::nothrow) uint32_t[masks.size()];
+    p->d.host_heads = new (std::nothrow) uint32_t[L.heads.size()];
+    if (!p->d.host_masks || !p->d.host_heads) {
+        delete[] p->d.host_masks;
+        delete[] p->d.host_heads;
+        delete p;
+        return DAMP_ERR_INVALID_ARGUMENT;
+    }
+    memcpy(p->d.host_masks, masks.data(), masks.size() * 4);
+    memcpy(p->d.host_heads, L.heads.data(), L.heads.size() * 4);
+    if (dev_buf) {
+        std::vector<uint8_t> hdr(d.header_bytes, 0);
+        memcpy(hdr.data() + damp::kStatusBytes, masks.data(), masks.size() * 4);
+        memcpy(hdr.data() + d.head_off, L.heads.data(), L.heads.size() * 4);
+        if (format != DAMP_FMT_FP32) {
+            // row directory: offsets of each key row (and its scale) in its head's block
+            uint32_t* dir = reinterpret_cast<uint32_t*>(hdr.data() + d.dir_off);
+            for (int h = 0; h < H; ++h) {
+                const uint32_t f16_off = L.heads[(size_t)h * 4 + 2];
+                const uint32_t i8_off = L.heads[(size_t)h * 4 + 3];
+                uint32_t r16 = 0, r8 = 0;
+                for (int i = 0; i < d_k; ++i) {
+                    const bool f16 = (masks[(size_t)h * damp::kMaskWords + (i >> 5)] >> (i & 31)) & 1u;
+                    uint32_t e;
+                    if (f16) {
+                        e = (f16_off + r16 * 2u * d_k) | (1u << 31);
+                        ++r16;
+                    } else {
+                        e = (i8_off + r8 * (uint32_t)d_k) | ((4u * r8) << 16);
+                        ++r8;
+                    }
+                    dir[(size_t)h * damp::kDirWords + i] = e;
+                }
+            }
+        }
+        cudaError_t e = cudaMemcpy(dev_buf, hdr.data(), hdr.size(), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = damp::prepare_decode(d);
+        if (e != cudaSuccess) {
+            delete[] p->d.host_masks;
+            delete[] p->d.host_heads;
+            delete p;
+            return DAMP_ERR_CUDA;
+        }
+    }
+    *out = p;
+    return DAMP_OK;
+}
+
+}  // namespace
+
+extern "C" {
 
 int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
                      const uint16_t* hp_row_idx, void* dev_buf, size_t buf_bytes,
@@ -119,66 +252,65 @@ int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_ro
             if (w & (1u << (i & 31))) return DAMP_ERR_INVALID_ARGUMENT;  // repeated row
             w |= 1u << (i & 31);
         }
-    PoolDesc d{};
-    d.format = format;
-    d.n_slots = n_slots;
-    d.H = H;
-    d.d = d_k;
-    d.hp = hp_rows;
-    layout(format, d_k, hp_rows, &d.block_bytes, &d.block_stride, &d.f16_off, &d.i8_off);
-    d.header_bytes = header_bytes(H);
-    d.dir_off = damp::dir_offset(H);
-    d.pool_bytes = d.header_bytes + (size_t)n_slots * H * d.block_stride;
-    if (dev_buf) {
-        if (!aligned16(dev_buf)) return DAMP_ERR_MISALIGNED;
-        if (buf_bytes < d.pool_bytes) return DAMP_ERR_BUFFER_TOO_SMALL;
+    return create_common(format, n_slots, H, d_k, hp_rows, masks, dev_buf, buf_bytes, out);
+}
+
+int damp_pool_bytes_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is_fp16,
+                        size_t* bytes) {
+    if (!bytes || !is_fp16 || n_slots < 1 || H < 1) return DAMP_ERR_INVALID_ARGUMENT;
+    int rc = check_shape(DAMP_FMT_MIXED, d_k, d_v, 0);
+    if (rc) return rc;
+    std::vector<uint32_t> masks;
+    if ((rc = masks_from_map(H, d_k, is_fp16, &masks))) return rc;
+    const Layout L = pool_layout(DAMP_FMT_MIXED, H, d_k, masks);
+    *bytes = header_bytes(H) + (size_t)n_slots * L.slot_stride;
+    return DAMP_OK;
+}
+
+int damp_pool_create_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is_fp16,
+                         void* dev_buf, size_t buf_bytes, damp_pool** out) {
+    if (!out) return DAMP_ERR_INVALID_ARGUMENT;
+    *out = nullptr;
+    if (n_slots < 1 || H < 1 || !is_fp16) return DAMP_ERR_INVALID_ARGUMENT;
+    int rc = check_shape(DAMP_FMT_MIXED, d_k, d_v, 0);
+    if (rc) return rc;
+    std::vector<uint32_t> masks;
+    if ((rc = masks_from_map(H, d_k, is_fp16, &masks))) return rc;
+    // one FP16-row count for every head -> the same pool as damp_pool_create
+    int hp = -1;
+    for (int h = 0; h < H; ++h) {
+        int c = 0;
+        for (int w = 0; w < damp::kMaskWords; ++w)
+            c += __builtin_popcount(masks[(size_t)h * damp::kMaskWords + w]);
+        hp = (h == 0 || c == hp) ? c : -2;
     }
-    damp_pool* p = new (std::nothrow) damp_pool;
-    if (!p) return DAMP_ERR_INVALID_ARGUMENT;
-    p->d = d;
-    p->d.dev_buf = static_cast<uint8_t*>(dev_buf);
-    p->d.host_masks = new (std::nothrow) uint32_t[masks.size()];
-    if (!p->d.host_masks) {
-        delete p;
-        return DAMP_ERR_INVALID_ARGUMENT;
-    }
-    memcpy(p->d.host_masks, masks.data(), masks.size() * 4);
-    if (dev_buf) {
-        std::vector<uint8_t> hdr(d.header_bytes, 0);
-        memcpy(hdr.data() + damp::kStatusBytes, masks.data(), masks.size() * 4);
-        if (format != DAMP_FMT_FP32) {
-            // row directory: offsets of each key row (and its scale) in a block
-            uint32_t* dir = reinterpret_cast<uint32_t*>(hdr.data() + d.dir_off);
-            for (int h = 0; h < H; ++h) {
-                uint32_t r16 = 0, r8 = 0;
-                for (int i = 0; i < d_k; ++i) {
-                    const bool f16 = (masks[(size_t)h * damp::kMaskWords + (i >> 5)] >> (i & 31)) & 1u;
-                    uint32_t e;
-                    if (f16) {
-                        e = (d.f16_off + r16 * 2u * d_k) | (1u << 31);
-                        ++r16;
-                    } else {
-                        e = (d.i8_off + r8 * (uint32_t)d_k) | ((4u * r8) << 16);
-                        ++r8;
-                    }
-                    dir[(size_t)h * damp::kDirWords + i] = e;
-                }
-            }
-        }
-        const cudaError_t e = cudaMemcpy(dev_buf, hdr.data(), hdr.size(), cudaMemcpyHostToDevice);
-        if (e != cudaSuccess) {
-            delete[] p->d.host_masks;
-            delete p;
-            return DAMP_ERR_CUDA;
+    return create_common(DAMP_FMT_MIXED, n_slots, H, d_k, hp < 0 ? -1 : hp, masks, dev_buf,
+                         buf_bytes, out);
+}
+
+int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,
+                          size_t* block_stride, size_t* offset_in_slot) {
+    if (!pool || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    const uint32_t* e = d.host_heads + (size_t)h * 4;
+    if (block_bytes) {
+        if (d.format == DAMP_FMT_FP32) {
+            *block_bytes = (size_t)d.d * d.d * 4;
+        } else {
+            const size_t r = (size_t)(e[3] - e[2]) / (2 * (size_t)d.d);   // FP16 rows
+            const size_t r8 = (size_t)d.d - r;
+            *block_bytes = 4 * r8 + 2 * r * d.d + r8 * d.d;
         }
     }
-    *out = p;
+    if (block_stride) *block_stride = e[1];
+    if (offset_in_slot) *offset_in_slot = e[0];
     return DAMP_OK;
 }
 
 int damp_pool_destroy(damp_pool* pool) {
     if (!pool) return DAMP_OK;
     delete[] pool->d.host_masks;
+    delete[] pool->d.host_heads;
     delete pool;
     return DAMP_OK;
 }
@@ -187,7 +319,7 @@ int damp_pool_block_offset(const damp_pool* pool, int slot, int h, size_t* offse
     if (!pool || !offset) return DAMP_ERR_INVALID_ARGUMENT;
     const PoolDesc& d = pool->d;
     if (slot < 0 || slot >= d.n_slots || h < 0 || h >= d.H) return DAMP_ERR_INVALID_ARGUMENT;
-    *offset = d.header_bytes + ((size_t)slot * d.H + h) * d.block_stride;
+    *offset = d.header_bytes + (size_t)slot * d.slot_stride + d.host_heads[(size_t)h * 4];
     return DAMP_OK;
 }
 
@@ -208,10 +340,8 @@ static int codec_args(const damp_pool* pool, int n, const int32_t* slot_idx, con
     a->n = n;
     a->H = d.H;
     a->n_slots = d.n_slots;
-    a->hp = d.hp;
-    a->block_stride = (uint32_t)d.block_stride;
-    a->f16_off = d.f16_off;
-    a->i8_off = d.i8_off;
+    a->heads = reinterpret_cast<const uint4*>(d.dev_buf + d.head_off);
+    a->slot_stride = d.slot_stride;
     const int upi = 128 / d.d;
     a->n_items = (int)(((size_t)n * d.H + upi - 1) / upi);
     return DAMP_OK;
@@ -265,14 +395,77 @@ int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int 
     a.n = n;
     a.H = d.H;
     a.n_slots = d.n_slots;
-    a.hp = d.hp;
+    a.heads = reinterpret_cast<const uint4*>(d.dev_buf + d.head_off);
+    a.slot_stride = d.slot_stride;
     a.block_stride = (uint32_t)d.block_stride;
-    a.f16_off = d.f16_off;
-    a.i8_off = d.i8_off;
     const int upi = 128 / d.d;
     a.n_items = (int)(((size_t)n * d.H + upi - 1) / upi);
     return cuda_status(
         damp::launch_decode_step(d, a, in_dtype, gate, static_cast<cudaStream_t>(stream)));
+}
+
+size_t damp_calib_bytes(int H, int d_k) {
+    if (H <= 0 || d_k <= 0) return 0;
+    return (2 * (size_t)H * d_k + (size_t)H) * sizeof(double);
+}
+
+int damp_calib_accumulate(const damp_pool* pool, int n, const int32_t* slot_idx, int gate,
+                          const float* alpha, double* acc, void* stream) {
+    if (!pool || n < 0 || !pool->d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    if (d.format != DAMP_FMT_FP32) return DAMP_ERR_INVALID_ARGUMENT;
+    if (gate != DAMP_GATE_SCALAR && gate != DAMP_GATE_VECTOR) return DAMP_ERR_INVALID_ARGUMENT;
+    if (n == 0) return DAMP_OK;
+    if (!slot_idx || !alpha || !acc) return DAMP_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(slot_idx) & 3u) || (reinterpret_cast<uintptr_t>(alpha) & 3u) ||
+        (reinterpret_cast<uintptr_t>(acc) & 7u))
+        return DAMP_ERR_MISALIGNED;
+    damp::CalibArgs a{};
+    a.state = reinterpret_cast<const float*>(d.dev_buf + d.header_bytes);
+    a.status = reinterpret_cast<uint32_t*>(d.dev_buf);
+    a.slot_idx = slot_idx;
+    a.alpha = alpha;
+    a.acc = acc;
+    a.n = n;
+    a.H = d.H;
+    a.n_slots = d.n_slots;
+    a.gate = gate;
+    return cuda_status(damp::launch_calib_accumulate(a, d.d, static_cast<cudaStream_t>(stream)));
+}
+
+static int calib_shape(int H, int d_k) {
+    if (H <= 0 || d_k <= 0) return DAMP_ERR_INVALID_ARGUMENT;
+    if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return DAMP_ERR_UNSUPPORTED;
+    return DAMP_OK;
+}
+
+int damp_calib_select(int H, int d_k, int hp_rows, const double* acc, double* score,
+                      uint16_t* hp_row_idx, void* stream) {
+    int rc = calib_shape(H, d_k);
+    if (rc) return rc;
+    if (hp_rows < 0 || hp_rows > d_k || !acc || (hp_rows > 0 && !hp_row_idx))
+        return DAMP_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(acc) & 7u) || (reinterpret_cast<uintptr_t>(score) & 7u) ||
+        (reinterpret_cast<uintptr_t>(hp_row_idx) & 1u))
+        return DAMP_ERR_MISALIGNED;
+    return cuda_status(damp::launch_calib_select(acc, H, d_k, hp_rows, score, hp_row_idx,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+int damp_calib_select_budget(int H, int d_k, int budget, const double* acc, double* score,
+                             uint8_t* is_fp16, int32_t* hp_per_head, void* stream) {
+    int rc = calib_shape(H, d_k);
+    if (rc) return rc;
+    if (budget < 0 || (size_t)budget > (size_t)H * d_k || !acc || !score || !is_fp16 ||
+        !hp_per_head)
+        return DAMP_ERR_INVALID_ARGUMENT;
+    if ((size_t)H * d_k > (size_t)0x7fffffff) return DAMP_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(acc) & 7u) || (reinterpret_cast<uintptr_t>(score) & 7u) ||
+        (reinterpret_cast<uintptr_t>(hp_per_head) & 3u))
+        return DAMP_ERR_MISALIGNED;
+    return cuda_status(damp::launch_calib_select_budget(acc, H, d_k, budget, score, is_fp16,
+                                                        hp_per_head,
+                                                        static_cast<cudaStream_t>(stream)));
 }
 
 int damp_pool_get_error(const damp_pool* pool, uint32_t* flags, int clear, void* stream) {
@@ -300,16 +493,17 @@ int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float
         return DAMP_OK;
     }
     if (!scale || !half || !code) return DAMP_ERR_INVALID_ARGUMENT;
+    const uint32_t f16_off = d.host_heads[(size_t)h * 4 + 2], i8_off = d.host_heads[(size_t)h * 4 + 3];
     int r16 = 0, r8 = 0;
     for (int i = 0; i < D; ++i) {
         if (is_fp16_row(d, h, i)) {
             scale[i] = 0.0f;
-            memcpy(half + (size_t)i * D, b + d.f16_off + (size_t)r16 * 2 * D, (size_t)2 * D);
+            memcpy(half + (size_t)i * D, b + f16_off + (size_t)r16 * 2 * D, (size_t)2 * D);
             memset(code + (size_t)i * D, 0, D);
             ++r16;
         } else {
             memcpy(&scale[i], b + (size_t)r8 * 4, 4);
-            memcpy(code + (size_t)i * D, b + d.i8_off + (size_t)r8 * D, D);
+            memcpy(code + (size_t)i * D, b + i8_off + (size_t)r8 * D, D);
             memset(half + (size_t)i * D, 0, (size_t)2 * D);
             ++r8;
         }
@@ -330,15 +524,16 @@ int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
         return DAMP_OK;
     }
     if (!scale || !half || !code) return DAMP_ERR_INVALID_ARGUMENT;
-    memset(b, 0, d.block_stride);
+    const uint32_t f16_off = d.host_heads[(size_t)h * 4 + 2], i8_off = d.host_heads[(size_t)h * 4 + 3];
+    memset(b, 0, d.host_heads[(size_t)h * 4 + 1]);
     int r16 = 0, r8 = 0;
     for (int i = 0; i < D; ++i) {
         if (is_fp16_row(d, h, i)) {
-            memcpy(b + d.f16_off + (size_t)r16 * 2 * D, half + (size_t)i * D, (size_t)2 * D);
+            memcpy(b + f16_off + (size_t)r16 * 2 * D, half + (size_t)i * D, (size_t)2 * D);
             ++r16;
         } else {
             memcpy(b + (size_t)r8 * 4, &scale[i], 4);
-            memcpy(b + d.i8_off + (size_t)r8 * D, code + (size_t)i * D, D);
+            memcpy(b + i8_off + (size_t)r8 * D, code + (size_t)i * D, D);
             ++r8;
         }
     }

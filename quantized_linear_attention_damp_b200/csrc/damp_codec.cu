@@ -24,7 +24,7 @@ namespace {
 
 constexpr int kCodecThreads = 256;
 
-template <int D, bool QUANT, bool PACK>
+template <int D, bool QUANT, bool PACK, bool FP8>
 __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a) {
     using G = Geo<D>;
     constexpr int RPT = G::RPT, UPI = G::UPI, LPR = G::LPR;
@@ -43,7 +43,9 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
         float* st = a.state + (size_t)u * D * D;
         const bool ok = slot >= 0 && slot < a.n_slots;
         if (!ok && slot >= a.n_slots && tu == 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
-        uint8_t* blk = ok ? a.blocks + ((size_t)slot * a.H + h) * (size_t)a.block_stride : nullptr;
+        // this head's block: {offset in the slot, stride, FP16-row offset, INT8-row offset}
+        const uint4 hb = __ldg(a.heads + h);
+        uint8_t* blk = ok ? a.blocks + (size_t)slot * a.slot_stride + hb.x : nullptr;
         uint32_t bits = 0;
         int rank16 = 0;
         if (QUANT && ok) {
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
                 x[i][1] = make_float2(f.z, f.w);
             }
             if constexpr (QUANT) {
-                store_quant_tile<D>(blk, a.f16_off, a.i8_off, bits, rank16, r0, cg, x, rowbuf);
+                store_quant_tile<D, FP8>(blk, hb.z, hb.w, bits, rank16, r0, cg, x, rowbuf);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i)
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
                 continue;
             }
             if constexpr (QUANT) {
-                load_quant_tile<D>(blk, a.f16_off, a.i8_off, bits, rank16, r0, cg, x);
+                load_quant_tile<D, FP8>(blk, hb.z, hb.w, bits, rank16, r0, cg, x);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
     }
 }
 
-template <int D, bool QUANT, bool PACK>
+template <int D, bool QUANT, bool PACK, bool FP8>
 cudaError_t launch_codec_t(const CodecArgs& a, cudaStream_t stream) {
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -103,18 +105,24 @@ cudaError_t launch_codec_t(const CodecArgs& a, cudaStream_t stream) {
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
     const int grid = std::max(1, std::min(a.n_items, sms * 8));
-    codec_kernel<D, QUANT, PACK><<<grid, kCodecThreads, 0, stream>>>(a);
+    codec_kernel<D, QUANT, PACK, FP8><<<grid, kCodecThreads, 0, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <int D, bool PACK>
+cudaError_t dispatch_d(int format, const CodecArgs& a, cudaStream_t s) {
+    if (format == DAMP_FMT_FP32) return launch_codec_t<D, false, PACK, false>(a, s);
+    if (format == DAMP_FMT_FP8_ROW) return launch_codec_t<D, true, PACK, true>(a, s);
+    return launch_codec_t<D, true, PACK, false>(a, s);
 }
 
 template <bool PACK>
 cudaError_t dispatch(const PoolDesc& p, const CodecArgs& a, cudaStream_t s) {
-    const bool q = p.format != DAMP_FMT_FP32;
     switch (p.d) {
-        case 16: return q ? launch_codec_t<16, true, PACK>(a, s) : launch_codec_t<16, false, PACK>(a, s);
-        case 32: return q ? launch_codec_t<32, true, PACK>(a, s) : launch_codec_t<32, false, PACK>(a, s);
-        case 64: return q ? launch_codec_t<64, true, PACK>(a, s) : launch_codec_t<64, false, PACK>(a, s);
-        case 128: return q ? launch_codec_t<128, true, PACK>(a, s) : launch_codec_t<128, false, PACK>(a, s);
+        case 16: return dispatch_d<16, PACK>(p.format, a, s);
+        case 32: return dispatch_d<32, PACK>(p.format, a, s);
+        case 64: return dispatch_d<64, PACK>(p.format, a, s);
+        case 128: return dispatch_d<128, PACK>(p.format, a, s);
         default: return cudaErrorInvalidValue;
     }
 }

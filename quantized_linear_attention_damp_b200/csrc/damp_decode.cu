@@ -65,7 +65,7 @@ __device__ __forceinline__ float bf16_at(const uint32_t* w, int i) {
     return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
 }
 
-template <int D, bool QUANT, bool KDA, bool BF16>
+template <int D, bool QUANT, bool KDA, bool BF16, bool FP8>
 __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs a) {
     using G = Geo<D>;
     constexpr int RPT = G::RPT, UPI = G::UPI, LPR = G::LPR;
@@ -124,10 +124,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         const int rel = (lane - il * UPI) & 31;
         if (rel < UPI) ring = load_meta(il * UPI + rel + 32);
         const bool load = lane < UPI && m.exists && m.slot >= 0 && m.slot < a.n_slots;
+        const int item_l = (int)blockIdx.x + il * (int)gridDim.x;
+        const int h_l = (item_l * UPI + lane) % a.H;
+        // this head's block: offset inside the slot and size (heads may differ)
+        const uint2 hb = load ? __ldg(reinterpret_cast<const uint2*>(a.heads + h_l)) : make_uint2(0u, 0u);
         uint32_t tx = 0;
         if (lane < UPI) {
             *reinterpret_cast<Meta*>(st + a.st_meta + lane * sizeof(Meta)) = m;
-            if (load) tx = a.block_stride + 3u * D * ELT + (KDA ? 4u * D : 0u) + (QUANT ? 4u * D : 0u);
+            if (load) tx = hb.y + 3u * D * ELT + (KDA ? 4u * D : 0u) + (QUANT ? 4u * D : 0u);
         }
         const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
         __syncwarp();
@@ -142,8 +146,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             const int h = u % a.H;
             const uint32_t fb = full_bar(stage);
             bulk_g2s(smem_u32(st + lane * a.block_stride),
-                     a.blocks + ((size_t)m.slot * a.H + h) * (size_t)a.block_stride,
-                     a.block_stride, fb);
+                     a.blocks + (size_t)m.slot * a.slot_stride + hb.x, hb.y, fb);
             const size_t io = (size_t)u * D * ELT;
             bulk_g2s(smem_u32(st + a.st_q + lane * D * ELT), static_cast<const uint8_t*>(a.q) + io,
                      D * ELT, fb);
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             }
             // ---- step 1: reconstruct S^
             if constexpr (QUANT) {
-                load_tile_dir<D>(blk, sdir, r0, cg, x);
+                load_tile_dir<D, FP8>(blk, sdir, r0, cg, x);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
                 x[i][1] = __ffma2_rn(f2(b), d1, x[i][1]);
             }
             if constexpr (QUANT) {
-                store_tile_dir<D>(blk, sdir, r0, cg, x, rowbuf);
+                store_tile_dir<D, FP8>(blk, sdir, r0, cg, x, rowbuf);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i)
@@ -342,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
                 const Meta m = *reinterpret_cast<const Meta*>(st + a.st_meta + w * sizeof(Meta));
                 if (m.exists && m.slot >= 0 && m.slot < a.n_slots) {
                     const int uw = item * UPI + w;
-                    uint8_t* gblk = a.blocks + ((size_t)m.slot * a.H + uw % a.H) *
-                                                   (size_t)a.block_stride;
-                    bulk_s2g(gblk, smem_u32(st + w * a.block_stride), a.block_stride);
+                    const uint2 hb = __ldg(reinterpret_cast<const uint2*>(a.heads + uw % a.H));
+                    bulk_s2g(a.blocks + (size_t)m.slot * a.slot_stride + hb.x,
+                             smem_u32(st + w * a.block_stride), hb.y);
                 }
             }
             bulk_commit();
@@ -398,11 +401,13 @@ Layout stage_layout(int d, uint32_t stride, int in_dtype, int gate) {
     return L;
 }
 
-template <int D, bool QUANT, bool KDA, bool BF16>
-cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
+// Kernel attributes are set once per instantiation (at pool creation, so that a
+// later launch can be captured into a CUDA graph with no set-up call inside).
+template <int D, bool QUANT, bool KDA, bool BF16, bool FP8>
+cudaError_t attrs_t() {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
-    auto kern = decode_step_kernel<D, QUANT, KDA, BF16>;
+    auto kern = decode_step_kernel<D, QUANT, KDA, BF16, FP8>;
     std::call_once(once, [&] {
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         227 * 1024);
@@ -410,6 +415,13 @@ cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
             attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                             100);
     });
+    return attr_err;
+}
+
+template <int D, bool QUANT, bool KDA, bool BF16, bool FP8>
+cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
+    auto kern = decode_step_kernel<D, QUANT, KDA, BF16, FP8>;
+    const cudaError_t attr_err = attrs_t<D, QUANT, KDA, BF16, FP8>();
     if (attr_err != cudaSuccess) return attr_err;
 
     StepArgs a = a0;
@@ -458,24 +470,67 @@ cudaError_t launch_t(const StepArgs& a0, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// Codec of the byte rows: 0 = FP32 state (no byte rows), 1 = INT8, 2 = FP8 E4M3.
+template <int D, int CODEC>
+cudaError_t dispatch_codec(const StepArgs& a, int in_dtype, int gate, cudaStream_t s) {
+    constexpr bool Q = CODEC != 0, F8 = CODEC == 2;
+    const bool kda = gate == DAMP_GATE_VECTOR, bf = in_dtype == DAMP_DTYPE_BF16;
+    if (kda) return bf ? launch_t<D, Q, true, true, F8>(a, s) : launch_t<D, Q, true, false, F8>(a, s);
+    return bf ? launch_t<D, Q, false, true, F8>(a, s) : launch_t<D, Q, false, false, F8>(a, s);
+}
+
+inline int codec_of(int format) {
+    return format == DAMP_FMT_FP32 ? 0 : format == DAMP_FMT_FP8_ROW ? 2 : 1;
+}
+
 template <int D>
 cudaError_t dispatch_fmt(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                          cudaStream_t s) {
-    const bool q = p.format != DAMP_FMT_FP32, kda = gate == DAMP_GATE_VECTOR,
-               bf = in_dtype == DAMP_DTYPE_BF16;
-    if (q) {
-        if (kda) return bf ? launch_t<D, true, true, true>(a, s) : launch_t<D, true, true, false>(a, s);
-        return bf ? launch_t<D, true, false, true>(a, s) : launch_t<D, true, false, false>(a, s);
+    switch (codec_of(p.format)) {
+        case 0: return dispatch_codec<D, 0>(a, in_dtype, gate, s);
+        case 2: return dispatch_codec<D, 2>(a, in_dtype, gate, s);
+        default: return dispatch_codec<D, 1>(a, in_dtype, gate, s);
     }
-    if (kda) return bf ? launch_t<D, false, true, true>(a, s) : launch_t<D, false, true, false>(a, s);
-    return bf ? launch_t<D, false, false, true>(a, s) : launch_t<D, false, false, false>(a, s);
+}
+
+template <int D, int CODEC>
+cudaError_t prepare_codec() {
+    constexpr bool Q = CODEC != 0, F8 = CODEC == 2;
+    cudaError_t e;
+    if ((e = attrs_t<D, Q, false, false, F8>()) != cudaSuccess) return e;
+    if ((e = attrs_t<D, Q, false, true, F8>()) != cudaSuccess) return e;
+    if ((e = attrs_t<D, Q, true, false, F8>()) != cudaSuccess) return e;
+    return attrs_t<D, Q, true, true, F8>();
+}
+
+template <int D>
+cudaError_t prepare_d(int codec) {
+    switch (codec) {
+        case 0: return prepare_codec<D, 0>();
+        case 2: return prepare_codec<D, 2>();
+        default: return prepare_codec<D, 1>();
+    }
 }
 
 }  // namespace
 
+cudaError_t prepare_decode(const PoolDesc& p) {
+    const int c = codec_of(p.format);
+    cudaError_t e;
+    switch (p.d) {
+        case 16: return prepare_d<16>(c);
+        case 32: return prepare_d<32>(c);
+        case 64: return prepare_d<64>(c);
+        case 128:
+            if ((e = prepare_d<128>(c)) != cudaSuccess) return e;
+            return c == 1 ? prepare_decode_pair() : cudaSuccess;
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream) {
-    if (p.d == 128 && p.format != DAMP_FMT_FP32 && decode_pair_fits(a, in_dtype, gate)) {
+    if (p.d == 128 && codec_of(p.format) == 1 && decode_pair_fits(a, in_dtype, gate)) {
         StepArgs b = a;
         b.n_items = ((a.n + 1) / 2) * a.H;   // pairs of batch entries x heads
         return launch_decode_pair(b, in_dtype, gate, stream);

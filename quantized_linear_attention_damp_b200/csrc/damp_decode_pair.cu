@@ -38,10 +38,10 @@ constexpr int kPG = 16;        // row groups (warps)
 // Per-unit metadata written by the issue warp into the stage (32 bytes).
 struct PMeta {
     int active;        // 1: block loaded, to be updated and stored
-    int exists;        // 1: the pair has this batch entry (out row to write)
+    uint32_t bytes;    // block size of the unit's head
     float alpha;       // GDN scalar decay
     float beta;
-    long long unit;    // b*H + h: row of q/k/v/alpha/beta/out
+    long long unit;    // b*H + h: row of q/k/v/alpha/beta/out; -1: no such entry
     long long boff;    // byte offset of the block in the pool; -1 if none
 };
 static_assert(sizeof(PMeta) == 32, "PMeta layout");
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     // U == L (mod 32), loaded 32 units ahead of use.
     constexpr int kIssueWarp = kPT / 32 - 1;
     auto load_meta = [&](int U) {
-        PMeta m{0, 0, 0.f, 0.f, 0, -1};
+        PMeta m{0, 0u, 0.f, 0.f, -1, -1};
         if (U < my_units) {
             const int g = (int)blockIdx.x + (U >> 1) * (int)gridDim.x;  // item: pair p, head h
             const int p = g / H, h = g - p * H;
@@ -110,13 +110,14 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
             if (b < a.n) {
                 const long long u = (long long)b * H + h;
                 const int slot = __ldg(a.slot_idx + b);
-                m.exists = 1;
                 m.unit = u;
                 if constexpr (!KDA) m.alpha = __ldg(a.alpha + u);
                 m.beta = __ldg(a.beta + u);
                 if (slot >= 0 && slot < a.n_slots) {
+                    const uint2 hb = __ldg(reinterpret_cast<const uint2*>(a.heads + h));
                     m.active = 1;
-                    m.boff = ((long long)slot * H + h) * (long long)a.block_stride;
+                    m.bytes = hb.y;
+                    m.boff = (long long)slot * (long long)a.slot_stride + hb.x;
                 } else if (slot >= a.n_slots) {
                     m.active = -1;   // out of range: flagged by the consumer
                 }
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         }
         return m;
     };
-    PMeta ring{0, 0, 0.f, 0.f, 0, -1};
+    PMeta ring{0, 0u, 0.f, 0.f, -1, -1};
     if (warp == kIssueWarp) ring = load_meta(lane);
 
     auto issue = [&](int il) {
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         const int src = (2 * il + lane) & 31;
         PMeta m;
         m.active = __shfl_sync(0xffffffffu, ring.active, src);
-        m.exists = __shfl_sync(0xffffffffu, ring.exists, src);
+        m.bytes = __shfl_sync(0xffffffffu, ring.bytes, src);
         m.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
         m.beta = __shfl_sync(0xffffffffu, ring.beta, src);
         m.unit = __shfl_sync(0xffffffffu, ring.unit, src);
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         uint32_t tx = 0;
         if (lane < 2) {
             *reinterpret_cast<PMeta*>(st + a.st_meta + lane * sizeof(PMeta)) = m;
-            if (load) tx = a.block_stride + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u);
+            if (load) tx = m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u);
             if (lane == 0 && loads) tx += 4u * kPD;   // the head's row directory
         }
         const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         __syncwarp();
         const uint32_t fb = full_bar(stage);
         if (load) {
-            bulk_g2s(smem_u32(st + lane * a.block_stride), a.blocks + m.boff, a.block_stride, fb);
+            bulk_g2s(smem_u32(st + lane * a.block_stride), a.blocks + m.boff, m.bytes, fb);
             const size_t io = (size_t)m.unit * kPD * ELT;
             bulk_g2s(smem_u32(st + a.st_q + lane * kPD * ELT),
                      static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
@@ -334,7 +335,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 const float dj = __fsub_rn(vj, uj);
                 delta_s[cu_ * kPD + j] = dj;
                 a.out[m.unit * kPD + j] = __fmaf_rn(c, dj, wj);
-            } else if (m.exists) {
+            } else if (m.unit >= 0) {
                 a.out[m.unit * kPD + j] = 0.f;
                 if (j == 0 && m.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
             }
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
             for (int w = 0; w < 2; ++w) {
                 const PMeta m = *reinterpret_cast<const PMeta*>(st + a.st_meta + w * sizeof(PMeta));
                 if (m.active == 1)
-                    bulk_s2g(a.blocks + m.boff, smem_u32(st + w * a.block_stride), a.block_stride);
+                    bulk_s2g(a.blocks + m.boff, smem_u32(st + w * a.block_stride), m.bytes);
             }
             bulk_commit();
         }
@@ -464,14 +465,20 @@ uint32_t pair_layout(StepArgs& a, bool kda, bool bf16) {
 }
 
 template <bool KDA, bool BF16>
-cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
+cudaError_t pair_attrs_t() {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
-    auto kern = decode_pair_kernel<KDA, BF16>;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        227 * 1024);
+        attr_err = cudaFuncSetAttribute(decode_pair_kernel<KDA, BF16>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     });
+    return attr_err;
+}
+
+template <bool KDA, bool BF16>
+cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
+    auto kern = decode_pair_kernel<KDA, BF16>;
+    const cudaError_t attr_err = pair_attrs_t<KDA, BF16>();
     if (attr_err != cudaSuccess) return attr_err;
     StepArgs a = a0;
     int dev = 0, sms = 0;
@@ -488,6 +495,14 @@ cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t prepare_decode_pair() {
+    cudaError_t e;
+    if ((e = pair_attrs_t<false, false>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<false, true>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<true, false>()) != cudaSuccess) return e;
+    return pair_attrs_t<true, true>();
+}
 
 bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate) {
     StepArgs b = a;

@@ -219,19 +219,45 @@ __device__ __forceinline__ float rowgroup_max(float m) {
     }
 }
 
-// scale = fl(a/127), inv = fl(127/a); zero / overflowing rows -> 0, 0.
+// scale = fl(a/Q), inv = fl(Q/a) with Q = 127 (INT8 rows) or 448 (the largest
+// finite FP8 E4M3 value); zero / overflowing rows -> 0, 0.
+template <bool FP8 = false>
 __device__ __forceinline__ void row_scale(float a, float& scale, float& inv) {
-    inv = __fdiv_rn(127.0f, a);
-    scale = __fdiv_rn(a, 127.0f);
+    constexpr float Q = FP8 ? 448.0f : 127.0f;
+    inv = __fdiv_rn(Q, a);
+    scale = __fdiv_rn(a, Q);
     if (a == 0.0f || isinf(inv)) {
         inv = 0.0f;
         scale = 0.0f;
     }
 }
 
+// fl(value(code) * s) for 4 FP8 E4M3 codes (byte j = element j).  Each pair
+// of codes is widened exactly to two FP16 values (E4M3 is a subset of FP16),
+// then to FP32, then scaled.
+__device__ __forceinline__ void dequant_e4m3x4(uint32_t w, float s, float2& lo, float2& hi) {
+    uint32_t h01, h23;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"((unsigned short)(w & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"((unsigned short)(w >> 16)));
+    lo = mul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&h01)), f2(s));
+    hi = mul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&h23)), f2(s));
+}
+
+// E4M3 codes of 4 values: the FP32 products x*inv converted to the nearest
+// E4M3 value (ties to even), saturating at +-448.  The conversion puts its
+// first source operand in the upper byte.
+__device__ __forceinline__ uint32_t quant_e4m3x4(float2 lo, float2 hi, float inv) {
+    const float2 a = mul2_rn(lo, f2(inv));
+    const float2 b = mul2_rn(hi, f2(inv));
+    unsigned short p01, p23;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(p01) : "f"(a.y), "f"(a.x));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(p23) : "f"(b.y), "f"(b.x));
+    return (uint32_t)p01 | ((uint32_t)p23 << 16);
+}
+
 // Load rows [r0, r0+RPT) x cols [4cg, 4cg+4) of a quantized block into x
 // (dequantized, not decayed).
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void load_quant_tile(const uint8_t* blk, uint32_t f16_off,
                                                 uint32_t i8_off, uint32_t bits, int rank16,
                                                 int r0, int cg, float2 (&x)[Geo<D>::RPT][2]) {
@@ -248,7 +274,8 @@ __device__ __forceinline__ void load_quant_tile(const uint8_t* blk, uint32_t f16
             const uint32_t w =
                 *reinterpret_cast<const uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4);
             const float s = *reinterpret_cast<const float*>(blk + (size_t)r8 * 4);
-            dequant_int8x4(w, s, x[i][0], x[i][1]);
+            if constexpr (FP8) dequant_e4m3x4(w, s, x[i][0], x[i][1]);
+            else dequant_int8x4(w, s, x[i][0], x[i][1]);
             ++r8;
         }
     }
@@ -257,7 +284,7 @@ __device__ __forceinline__ void load_quant_tile(const uint8_t* blk, uint32_t f16
 // Requantize rows [r0, r0+RPT) of x into a quantized block at `blk` (shared or
 // global).  rowbuf: 2*RPT floats private to this row group (shared memory).
 // Must be called by every lane of the warp (it synchronises the warp).
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off, uint32_t i8_off,
                                                  uint32_t bits, int rank16, int r0, int cg,
                                                  const float2 (&x)[Geo<D>::RPT][2],
@@ -277,7 +304,7 @@ __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off,
     __syncwarp();
     if (cg < RPT && !((bits >> cg) & 1u)) {
         float scale, inv;
-        row_scale(rowbuf[cg], scale, inv);
+        row_scale<FP8>(rowbuf[cg], scale, inv);
         rowbuf[RPT + cg] = inv;
         const int rank8 = r0 + cg - rank16 - __popc(bits & ((1u << cg) - 1u));
         *reinterpret_cast<float*>(blk + (size_t)rank8 * 4) = scale;
@@ -292,7 +319,8 @@ __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off,
             ++r16;
         } else {
             *reinterpret_cast<uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4) =
-                quant_int8x4(x[i][0], x[i][1], rowbuf[RPT + i]);
+                FP8 ? quant_e4m3x4(x[i][0], x[i][1], rowbuf[RPT + i])
+                    : quant_int8x4(x[i][0], x[i][1], rowbuf[RPT + i]);
             ++r8;
         }
     }
@@ -324,7 +352,7 @@ __device__ __forceinline__ float absmax4_3(float2 lo, float2 hi) {
     return fmaxf(m, fabsf(hi.y));
 }
 
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void load_tile_dir(const uint8_t* blk, const uint32_t* dir, int r0,
                                               int cg, float2 (&x)[Geo<D>::RPT][2]) {
     constexpr int RPT = Geo<D>::RPT;
@@ -346,12 +374,13 @@ __device__ __forceinline__ void load_tile_dir(const uint8_t* blk, const uint32_t
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
             if (e[j] >> 31) dequant_fp16x4(w16[j], x[i0 + j][0], x[i0 + j][1]);
+            else if constexpr (FP8) dequant_e4m3x4(w8[j], sc[j], x[i0 + j][0], x[i0 + j][1]);
             else dequant_int8x4_cvt(w8[j], sc[j], x[i0 + j][0], x[i0 + j][1]);
         }
     }
 }
 
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void store_tile_dir(uint8_t* blk, const uint32_t* dir, int r0, int cg,
                                                const float2 (&x)[Geo<D>::RPT][2],
                                                float* rowbuf) {
@@ -368,7 +397,7 @@ __device__ __forceinline__ void store_tile_dir(uint8_t* blk, const uint32_t* dir
         const uint32_t e = dir[r0 + cg];
         if (!(e >> 31)) {
             float scale, inv;
-            row_scale(rowbuf[cg], scale, inv);
+            row_scale<FP8>(rowbuf[cg], scale, inv);
             rowbuf[RPT + cg] = inv;
             *reinterpret_cast<float*>(blk + ((e >> 16) & 0x7fffu)) = scale;
         }
@@ -382,7 +411,8 @@ __device__ __forceinline__ void store_tile_dir(uint8_t* blk, const uint32_t* dir
             *reinterpret_cast<uint2*>(row + cg * 8) = quant_fp16x4(x[i][0], x[i][1]);
         } else {
             *reinterpret_cast<uint32_t*>(row + cg * 4) =
-                quant_int8x4(x[i][0], x[i][1], rowbuf[RPT + i]);
+                FP8 ? quant_e4m3x4(x[i][0], x[i][1], rowbuf[RPT + i])
+                    : quant_int8x4(x[i][0], x[i][1], rowbuf[RPT + i]);
         }
     }
     __syncwarp();

@@ -10,7 +10,11 @@ namespace damp {
 //   [0, 16)                      device status word (uint32) + padding
 //   [16, 16 + 16*H)              per-head FP16-row masks, 4 x uint32 (key rows 0..127)
 //   [dir_off, dir_off + 512*H)   per-head row directory, 128 x uint32 (see below)
-// rounded up to 256 bytes; the blocks follow.
+//   [head_off, head_off + 16*H)  per-head block table, uint4 {block offset inside
+//                                the slot, block stride, FP16-row offset, INT8-row
+//                                offset} (heads may hold different FP16-row counts)
+// rounded up to 256 bytes; the blocks follow, slot s at header + s*slot_stride,
+// head h of it at + table[h].x.
 //
 // Row directory entry of key row i of a quantized block:
 //   bits  0..15  byte offset of the row inside the block
@@ -21,15 +25,21 @@ constexpr int kMaskWords = 4;
 constexpr int kMaxD = 128;
 constexpr int kDirWords = 128;
 inline size_t dir_offset(int H) { return (kStatusBytes + (size_t)H * kMaskWords * 4 + 15) / 16 * 16; }
+inline size_t head_table_offset(int H) { return dir_offset(H) + (size_t)H * kDirWords * 4; }
 
 struct PoolDesc {
     int format;      // DAMP_FMT_*
-    int n_slots, H, d, hp;
-    size_t block_bytes, block_stride, header_bytes, pool_bytes;
-    uint32_t f16_off, i8_off;  // byte offsets inside a quantized block
+    int n_slots, H, d;
+    int hp;                    // FP16 rows per head; -1 when heads differ
+    size_t block_bytes;        // largest algorithmic block size over the heads
+    size_t block_stride;       // largest block stride over the heads (stage size)
+    size_t slot_stride;        // bytes of one slot (all its heads)
+    size_t header_bytes, pool_bytes;
     uint8_t* dev_buf;          // caller's buffer (NULL: host-only descriptor)
     uint32_t* host_masks;      // [H][kMaskWords]
+    uint32_t* host_heads;      // [H][4], as the header's block table
     size_t dir_off;            // byte offset of the row directory in the header
+    size_t head_off;           // byte offset of the block table in the header
 };
 
 // Arguments of the decode-step kernel.
@@ -45,9 +55,10 @@ struct StepArgs {
     const float* alpha;
     const float* beta;
     float* out;
-    int n, H, n_slots, hp;
-    uint32_t block_stride;     // bytes
-    uint32_t f16_off, i8_off;  // offsets inside a block
+    const uint4* heads;        // [H] block table (see the header layout)
+    unsigned long long slot_stride;
+    int n, H, n_slots;
+    uint32_t block_stride;     // largest block stride (stage buffer size)
     int n_items;               // work items (groups of 128/d units)
     int n_stages;
     // offsets inside one pipeline stage (bytes)
@@ -63,18 +74,39 @@ struct CodecArgs {
     uint32_t* status;
     const int32_t* slot_idx;
     float* state;              // [n][H][d][d]
-    int n, H, n_slots, hp;
-    uint32_t block_stride, f16_off, i8_off;
+    const uint4* heads;        // [H] block table
+    unsigned long long slot_stride;
+    int n, H, n_slots;
     int n_items;
 };
 
-// Launchers (damp_decode.cu, damp_codec.cu).  They return cudaError_t.
+// Arguments of the calibration accumulate kernel (damp_calib.cu).
+struct CalibArgs {
+    const float* state;        // first FP32 block of the pool
+    uint32_t* status;
+    const int32_t* slot_idx;
+    const float* alpha;
+    double* acc;               // energy [H][d], retention [H][d], count [H]
+    int n, H, n_slots, gate;
+};
+
+// Launchers (damp_decode.cu, damp_codec.cu, damp_calib.cu).  They return cudaError_t.
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream);
 // d = 128 quantized states, two units of one head per CTA iteration
 // (damp_decode_pair.cu); a.n_items counts pairs x heads.
 cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, cudaStream_t stream);
 bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate);   // >= 3 stages fit
+// One-time kernel attribute set-up for every decode variant a pool can launch
+// (called by damp_pool_create, outside any stream capture).
+cudaError_t prepare_decode(const PoolDesc& p);
+cudaError_t prepare_decode_pair();
+cudaError_t launch_calib_accumulate(const CalibArgs& a, int d, cudaStream_t stream);
+cudaError_t launch_calib_select(const double* acc, int H, int d, int hp, double* score,
+                                uint16_t* idx, cudaStream_t stream);
+cudaError_t launch_calib_select_budget(const double* acc, int H, int d, int budget,
+                                       double* score, uint8_t* is_fp16, int32_t* hp,
+                                       cudaStream_t stream);
 cudaError_t launch_pack(const PoolDesc& p, const CodecArgs& a, cudaStream_t stream);
 cudaError_t launch_unpack(const PoolDesc& p, const CodecArgs& a, cudaStream_t stream);
 

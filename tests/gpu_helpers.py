@@ -19,7 +19,7 @@ ATOL_OUT = 1e-5
 
 
 def oracle_fmt(fmt: str) -> int:
-    return O.FMT_FP32 if fmt == "fp32" else O.FMT_QUANT
+    return {"fp32": O.FMT_FP32, "fp8": O.FMT_FP8}.get(fmt, O.FMT_QUANT)
 
 
 def gate_of(w: W.Workload) -> int:
@@ -41,13 +41,18 @@ def torch_inputs(w: W.Workload, x: W.StepInputs, device="cuda") -> dict:
 class Pair:
     """A GPU pool and an oracle pool built from the same workload."""
 
-    def __init__(self, w: W.Workload, fmt: str | None = None, oracle_slots=None):
+    def __init__(self, w: W.Workload, fmt: str | None = None, oracle_slots=None,
+                 fp16_map=None):
         self.w = w
         self.fmt = fmt or w.fmt
         self.hs = W.head_structure(w.with_(fmt=self.fmt))
-        self.is_fp16 = self.hs.is_fp16
-        hp_idx = self.hs.hp_row_idx if self.fmt == "mixed" else None
-        self.gpu = D.DampPool(self.fmt, w.n_slots, w.H, w.d, hp_idx)
+        if fp16_map is not None:           # per-head FP16-row counts may differ
+            self.is_fp16 = np.ascontiguousarray(fp16_map, np.uint8)
+            self.gpu = D.DampPool("mixed", w.n_slots, w.H, w.d, fp16_map=self.is_fp16)
+        else:
+            self.is_fp16 = self.hs.is_fp16
+            hp_idx = self.hs.hp_row_idx if self.fmt == "mixed" else None
+            self.gpu = D.DampPool(self.fmt, w.n_slots, w.H, w.d, hp_idx)
         S0 = W.initial_state(w, range(w.n_slots))
         self.gpu.pack(torch.arange(w.n_slots, dtype=torch.int32, device="cuda"),
                       torch.from_numpy(S0).cuda())

@@ -67,6 +67,7 @@ def test_format_accounting_matches_published_figures():
 def test_layouts_of_other_formats():
     assert D.damp_layout(D.DAMP_FMT_FP32, 128, 128, 0) == (65536, 65536)
     assert D.damp_layout(D.DAMP_FMT_INT8_ROW, 128, 128, 0) == (16896, 16896)
+    assert D.damp_layout(D.DAMP_FMT_FP8_ROW, 128, 128, 0) == (16896, 16896)
     assert D.damp_layout(D.DAMP_FMT_MIXED, 128, 128, 0) == (16896, 16896)
     assert D.damp_layout(D.DAMP_FMT_MIXED, 128, 128, 128) == (32768, 32768)
     assert D.damp_layout(D.DAMP_FMT_MIXED, 16, 16, 4) == (368, 368)
@@ -78,13 +79,15 @@ def test_layouts_of_other_formats():
 
 def test_pool_bytes():
     n = D.damp_pool_bytes(D.DAMP_FMT_MIXED, 64, 32, 128, 128, 27)
-    # status word, 16-byte FP16-row mask and 512-byte row directory per head
-    hdr = 256 * ((16 + 32 * 16 + 32 * 512 + 255) // 256)
+    # status word; per head a 16-byte FP16-row mask, a 512-byte row directory
+    # and a 16-byte block-table entry
+    hdr = 256 * ((16 + 32 * 16 + 32 * 512 + 32 * 16 + 255) // 256)
     assert n == hdr + 64 * 32 * 20256
 
 
 @pytest.mark.parametrize("args,status", [
-    ((3, 128, 128, 0), D.DAMP_ERR_INVALID_ARGUMENT),         # bad format
+    ((4, 128, 128, 0), D.DAMP_ERR_INVALID_ARGUMENT),         # bad format
+    ((D.DAMP_FMT_FP8_ROW, 128, 128, 2), D.DAMP_ERR_INVALID_ARGUMENT),
     ((D.DAMP_FMT_MIXED, 128, 128, 129), D.DAMP_ERR_INVALID_ARGUMENT),
     ((D.DAMP_FMT_MIXED, 128, 128, -1), D.DAMP_ERR_INVALID_ARGUMENT),
     ((D.DAMP_FMT_INT8_ROW, 128, 128, 3), D.DAMP_ERR_INVALID_ARGUMENT),
@@ -174,3 +177,46 @@ def test_block_logical_round_trip(d, hp):
                                   .view(np.int8), code[~is16].reshape(-1))
     finally:
         D.damp_pool_destroy(h)
+
+
+def test_per_head_map_layout():
+    """Heads with different FP16-row counts: each head's block has the layout
+    of its own count, the slot is their concatenation, and a map with one
+    count everywhere is the fixed-count pool."""
+    d, H = 64, 4
+    g = np.random.default_rng(2)
+    counts = [0, 5, 64, 17]
+    m = np.zeros((H, d), np.uint8)
+    for h, c in enumerate(counts):
+        m[h, g.permutation(d)[:c]] = 1
+    h = D.damp_pool_create_map(3, H, d, d, m, None)
+    try:
+        off = 0
+        for head, c in enumerate(counts):
+            b, st, o = D.damp_pool_head_layout(h, head)
+            assert (b, st) == D.damp_layout(D.DAMP_FMT_MIXED, d, d, c) and o == off
+            off += st
+        hdr = D.damp_pool_block_offset(h, 0, 0)
+        assert D.damp_pool_block_offset(h, 2, 3) == hdr + 2 * off + D.damp_pool_head_layout(h, 3)[2]
+        assert D.damp_pool_bytes_map(3, H, d, d, m) == hdr + 3 * off
+        # logical round trip through the per-head layout
+        for head, c in enumerate(counts):
+            st = D.damp_pool_head_layout(h, head)[1]
+            is16 = m[head].astype(bool)
+            scale = np.where(is16, 0, g.uniform(0.1, 2, d)).astype(np.float32)
+            half = np.where(is16[:, None], g.integers(0, 0x7C00, (d, d)), 0).astype(np.uint16)
+            code = np.where(is16[:, None], 0, g.integers(-127, 128, (d, d))).astype(np.int8)
+            raw = D.damp_block_from_logical(h, head, st, scale=scale, half=half, code=code)
+            back = D.damp_block_to_logical(h, head, raw, D.DAMP_FMT_MIXED, d)
+            assert np.array_equal(back["half"], half) and np.array_equal(back["code"], code)
+            assert np.array_equal(back["scale"], scale)
+    finally:
+        D.damp_pool_destroy(h)
+    same = np.zeros((H, d), np.uint8)
+    same[:, :7] = 1
+    assert D.damp_pool_bytes_map(5, H, d, d, same) == \
+        D.damp_pool_bytes(D.DAMP_FMT_MIXED, 5, H, d, d, 7)
+    with pytest.raises(D.DampError):
+        bad = same.copy()
+        bad[0, 0] = 2
+        D.damp_pool_bytes_map(5, H, d, d, bad)

@@ -5,7 +5,8 @@ only) and the oracle from the same seeded inputs; each side keeps its own
 state.  States are expected bit-exact (each rounding is taken in the same
 precision and order on both sides); the asserted bar is the stated one:
 readouts within 1e-4 relative / 1e-5 absolute, FP16 rows and scales within
-1 ulp, INT8 codes within +-1 on at most 0.1 % of entries.
+1 ulp, INT8 codes within +-1 on at most 0.1 % of entries (FP8 E4M3 codes,
+a comparison format with no stated bar, are held to the same).
 """
 import numpy as np
 import pytest
@@ -37,8 +38,8 @@ SMALL = {
 }
 
 
-def run_full(w, fmt, steps):
-    p = Pair(w, fmt)
+def run_full(w, fmt, steps, fp16_map=None):
+    p = Pair(w, fmt, fp16_map=fp16_map)
     try:
         rep = p.check_state()
         assert rep["exact"], rep            # pack parity
@@ -61,7 +62,7 @@ def test_tiny_gdn_full_trajectory():
 
 
 @pytest.mark.parametrize("name", list(SMALL))
-@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp32"])
+@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp8", "fp32"])
 def test_small_shapes_all_formats(name, fmt):
     w = SMALL[name]
     run_full(w, fmt, min(w.steps, 8))
@@ -80,13 +81,40 @@ def test_all_fp16_rows_d128():
     run_full(w, "mixed", 3)
 
 
+def random_map(H, d, counts, seed):
+    g = np.random.default_rng(seed)
+    m = np.zeros((H, d), np.uint8)
+    for h, c in enumerate(counts):
+        m[h, g.permutation(d)[:c]] = 1
+    return m
+
+
+@pytest.mark.parametrize("name", ["tiny_kda", "d32_gdn_bf16", "d64_kda_bf16", "d128_ragged",
+                                  "d128_kda_f32"])
+def test_per_head_fp16_row_counts(name):
+    """Heads with different FP16-row counts (incl. none and all rows) in one
+    pool: per-head block layouts, per-head offsets inside a slot."""
+    w = SMALL[name]
+    base = [0, w.d, w.d // 3, 1, w.d - 1]
+    counts = [base[h % len(base)] for h in range(w.H)]
+    run_full(w, "mixed", min(w.steps, 4), fp16_map=random_map(w.H, w.d, counts, w.H * w.d))
+
+
+def test_per_head_fp16_row_counts_pair_kernel():
+    """d = 128 with every head's block small enough for the two-unit kernel's
+    stages (no all-FP16 head)."""
+    w = SMALL["d128_ragged"].with_(name="d128_varhp", H=6)
+    counts = [0, 27, 60, 1, 100, 27]
+    run_full(w, "mixed", 3, fp16_map=random_map(w.H, w.d, counts, 77))
+
+
 @pytest.mark.parametrize("name,steps", [("gdn_batch", 3), ("kda", 2)])
 def test_full_size_whole_state(name, steps):
     """The 64x32 GDN and 128x32 KDA workloads at full size, every unit compared."""
     run_full(W.WORKLOADS[name], "mixed", steps)
 
 
-@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp32"])
+@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp8", "fp32"])
 def test_high_concurrency_sampled_units(fmt):
     """512 slots x 48 heads at full size (the launch the benchmark times);
     sampled slots followed by the oracle over 4 steps."""

@@ -55,7 +55,7 @@ class Workload:
     steps: int
     gate: str         # "gdn" | "kda"
     in_dtype: str     # "bf16" | "f32"
-    fmt: str = "mixed"  # "mixed" | "int8" | "fp32"
+    fmt: str = "mixed"  # "mixed" | "int8" | "fp8" | "fp32"
     tiny: bool = False
     seed: int = 0
 
@@ -151,7 +151,7 @@ def head_structure(w: Workload) -> HeadStructure:
     is_fp16 = np.zeros((H, d), np.uint8)
     for h in range(H):
         is_fp16[h, hp_idx[h]] = 1
-    if w.fmt == "int8":
+    if w.fmt in ("int8", "fp8"):
         hp_idx = np.zeros((H, 0), np.uint16)
         is_fp16[:] = 0
     return HeadStructure(row_mult, col_mult, decay_a, tiny_alpha, hp_idx, is_fp16)
@@ -214,3 +214,39 @@ def step_inputs(w: Workload, step: int, hs: HeadStructure | None = None) -> Step
         vb, v = bf16_round(v)
     return StepInputs(slot_idx, q, k, v, qb, kb, vb, np.ascontiguousarray(alpha),
                       np.ascontiguousarray(beta))
+
+
+# ----------------------------------------------------------------------------
+# Serving-shaped slot pool: 36 GDN-family layers x 32 heads, d = 128, a pool of
+# 4096 slots per layer, and per step a random subset of 1024 slots (the same
+# requests in every layer).  Every fourth layer (index 3 mod 4) is a KDA layer
+# with per-key-channel decay.  To keep set-up tractable on the host, the
+# initial state of slot s is the state drawn for template slot s mod 64 of
+# that layer (64 templates per layer, each drawn as in initial_state).
+# ----------------------------------------------------------------------------
+
+SERVING_LAYERS = 36
+SERVING_TEMPLATES = 64
+
+
+def serving_layer(layer: int, seed: int = 0) -> Workload:
+    gate = GATE_KDA if layer % 4 == 3 else GATE_GDN
+    return Workload(f"serving_pool_l{layer}", n=1024, n_slots=4096, H=32, d=128, hp=27,
+                    steps=16, gate=gate, in_dtype="bf16", seed=seed)
+
+
+def serving_slot_idx(step: int, seed: int = 0, n: int = 1024, n_slots: int = 4096) -> np.ndarray:
+    """The step's batch: a random subset of n pool slots, shared by all layers."""
+    g = np.random.default_rng([seed, _tag("serving_pool"), _tag("slots"), step])
+    return g.permutation(n_slots)[:n].astype(np.int32)
+
+
+def serving_templates(w: Workload) -> np.ndarray:
+    """Template states [SERVING_TEMPLATES][H][d][d]; slot s starts as template s % 64."""
+    return initial_state(w, range(SERVING_TEMPLATES))
+
+
+def serving_step_inputs(w: Workload, step: int, hs: HeadStructure | None = None) -> StepInputs:
+    x = step_inputs(w, step, hs)
+    x.slot_idx = serving_slot_idx(step, w.seed, w.n, w.n_slots)
+    return x
