@@ -188,7 +188,8 @@ class Bench:
     serving pool much larger than L2 does.  No step is flushed or skipped.
     """
 
-    def __init__(self, w: W.Workload, fmt: str, device, n_inputs: int | None = None):
+    def __init__(self, w: W.Workload, fmt: str, device, n_inputs: int | None = None,
+                 fp16_map=None):
         import torch
 
         import quantized_linear_attention_damp_b200 as D
@@ -197,14 +198,17 @@ class Bench:
         self.hs = W.head_structure(w.with_(fmt=fmt))
         hp = self.hs.hp_row_idx if fmt == "mixed" else None
         l2 = torch.cuda.get_device_properties(device).L2_cache_size
-        _, stride = D.damp_layout(D.FORMATS[fmt], w.d, w.d, w.hp if fmt == "mixed" else 0)
-        state_bytes = w.n_slots * w.H * stride
+        if fp16_map is not None:
+            state_bytes = D.damp_pool_bytes_map(w.n_slots, w.H, w.d, w.d, fp16_map)
+        else:
+            _, stride = D.damp_layout(D.FORMATS[fmt], w.d, w.d, w.hp if fmt == "mixed" else 0)
+            state_bytes = w.n_slots * w.H * stride
         self.n_pools = max(1, -(-4 * l2 // state_bytes))
         S0 = torch.from_numpy(W.initial_state(w, range(w.n_slots))).to(device)
         ident = torch.arange(w.n_slots, dtype=torch.int32, device=device)
         self.pools = []
         for _ in range(self.n_pools):
-            p = D.DampPool(fmt, w.n_slots, w.H, w.d, hp, device=device)
+            p = D.DampPool(fmt, w.n_slots, w.H, w.d, hp, device=device, fp16_map=fp16_map)
             p.pack(ident, S0)
             self.pools.append(p)
         del S0
@@ -293,7 +297,7 @@ def cpu_baseline(w: W.Workload, fmt: str, seconds: float, max_units: int = 10 **
     """Oracle head-steps/s on one host core over a bounded sample of units."""
     import oracle as O
     hs = W.head_structure(w.with_(fmt=fmt))
-    ofmt = O.FMT_FP32 if fmt == "fp32" else O.FMT_QUANT
+    ofmt = {"fp32": O.FMT_FP32, "fp8": O.FMT_FP8}.get(fmt, O.FMT_QUANT)
     x = W.step_inputs(w, 0, hs)
     slots = list(x.slot_idx[: min(w.n, 8)])
     S0 = W.initial_state(w, slots)
@@ -368,6 +372,10 @@ def run_native(args, rank, world, local_rank):
                                           f"one step each, single thread, {el:.1f} s"}
     if world == 1 and not args.no_variants:
         line["variants"] = variants(args, dev)
+    if world == 1 and not args.no_variants:
+        line["state_error_vs_fp32"] = quality(dev)
+    if world == 1 and not args.no_serving:
+        line["serving_pool"] = serving(args, dev)
     print(json.dumps(line), flush=True)
 
 
@@ -376,8 +384,8 @@ def variants(args, dev):
     res = []
     steps = max(20, min(args.steps, 200))
     for name, fmt in [("gdn_256x32", "mixed"), ("kda", "mixed"), ("hiconc_gdn", "mixed"),
-                      ("hiconc_gdn", "int8"), ("hiconc_gdn", "fp32"), ("gdn_batch", "int8"),
-                      ("gdn_batch", "fp32")]:
+                      ("hiconc_gdn", "int8"), ("hiconc_gdn", "fp8"), ("hiconc_gdn", "fp32"),
+                      ("gdn_batch", "int8"), ("gdn_batch", "fp32")]:
         w = W.WORKLOADS[name]
         b = Bench(w, fmt, device=dev)
         secs = b.timed(steps, 3)
@@ -389,6 +397,228 @@ def variants(args, dev):
         res.append({"workload": describe(w, fmt), "head_steps_per_s": units * steps / secs,
                     "us_per_step": secs / steps * 1e6, "hbm_gbs": gbs, "frac": gbs / peak,
                     "bytes_per_unit": ub})
+    # pack / unpack at pool scale (prefill hand-off and restore): 512 x 48 units
+    import torch
+
+    import quantized_linear_attention_damp_b200 as D
+    w = W.WORKLOADS["hiconc_gdn"]
+    b = Bench(w, "mixed", device=dev, n_inputs=1)
+    units = w.n_slots * w.H
+    S = torch.empty((w.n_slots, w.H, w.d, w.d), dtype=torch.float32, device=dev)
+    ident = torch.arange(w.n_slots, dtype=torch.int32, device=dev)
+    for name_, fn in (("unpack", lambda p: p.unpack(ident, S)), ("pack", lambda p: p.pack(ident, S))):
+        for i in range(3):
+            fn(b.pools[i % b.n_pools])
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(10)]
+        for i in range(10):
+            ev[i][0].record()
+            fn(b.pools[i % b.n_pools])
+            ev[i][1].record()
+        torch.cuda.synchronize(dev)
+        secs = sum(a_.elapsed_time(b_) for a_, b_ in ev) / 1e3
+        # FP32 state (d*d*4) one way, the block's algorithmic bytes the other
+        ub = 4 * w.d * w.d + D.damp_layout(D.DAMP_FMT_MIXED, w.d, w.d, w.hp)[0]
+        gbs = ub * units * 10 / secs / 1e9
+        res.append({"workload": f"{name_}: {w.n_slots} slots x {w.H} heads, d={w.d}, mixed "
+                                f"({w.hp} FP16 rows/head) <-> FP32 states",
+                    "head_steps_per_s": units * 10 / secs, "us_per_step": secs / 10 * 1e6,
+                    "hbm_gbs": gbs, "frac": gbs / measured_peak()[0], "bytes_per_unit": ub})
+    b.close()
+    del S
+    # calibrated FP16 rows under one budget for all heads (counts differ per head)
+    w = W.WORKLOADS["gdn_256x32"]
+    acc = calibrate(w, dev)
+    is16, hp, _ = D.damp_calib_select_budget(w.H, w.d, w.hp * w.H, acc)
+    fmap = is16.cpu().numpy()
+    b = Bench(w, "mixed", device=dev, fp16_map=fmap)
+    secs = b.timed(steps, 3)
+    blk = [b.pools[0].heads[h][0] for h in range(w.H)]
+    b.close()
+    elt = 2 if w.in_dtype == "bf16" else 4
+    ub = 2 * float(np.mean(blk)) + 3 * w.d * elt + 4 + 4 + 4 * w.d
+    units = w.n * w.H
+    gbs = ub * units * steps / secs / 1e9
+    res.append({"workload": describe(w, "mixed").replace(
+                    f"({w.hp} FP16 rows/head)",
+                    f"(calibrated, {w.hp * w.H} FP16 rows over {w.H} heads, "
+                    f"{int(hp.min())}..{int(hp.max())} per head)"),
+                "head_steps_per_s": units * steps / secs, "us_per_step": secs / steps * 1e6,
+                "hbm_gbs": gbs, "frac": gbs / measured_peak()[0], "bytes_per_unit": ub})
+    return res
+
+
+def calibrate(w: W.Workload, dev, steps: int = 8):
+    """GPU calibration of the FP16-row choice on workload ``w``: the FP32
+    recurrence runs ``steps`` steps from the workload's initial state and
+    every step's states are recorded (damp_calib_accumulate)."""
+    import torch
+
+    import quantized_linear_attention_damp_b200 as D
+    hs = W.head_structure(w.with_(fmt="fp32"))
+    p = D.DampPool("fp32", w.n_slots, w.H, w.d, device=dev)
+    p.pack(torch.arange(w.n_slots, dtype=torch.int32, device=dev),
+           torch.from_numpy(W.initial_state(w, range(w.n_slots))).to(dev))
+    acc = D.calib_acc(w.H, w.d, device=dev)
+    out = torch.empty((w.n, w.H, w.d), dtype=torch.float32, device=dev)
+    for s in range(steps):
+        x = W.step_inputs(w.with_(name=w.name + "_calib"), s, hs)
+        cv = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        t = dict(slot_idx=torch.from_numpy(x.slot_idx).to(dev), q=cv(x.q_bits), k=cv(x.k_bits),
+                 v=cv(x.v_bits), alpha=torch.from_numpy(x.alpha).to(dev),
+                 beta=torch.from_numpy(x.beta).to(dev))
+        p.step(t["slot_idx"], t["q"], t["k"], t["v"], t["alpha"], t["beta"], out)
+        D.damp_calib_accumulate(p.handle, t["slot_idx"], t["alpha"], acc)
+    p.close()
+    return acc
+
+
+def quality(dev, steps: int = 64):
+    """Context: state error of each format after ``steps`` decode steps, as
+    the relative Frobenius distance of the dequantized state from the FP32
+    recurrence fed the same inputs (64 slots x 32 heads GDN and 128 x 32 KDA,
+    d = 128).  Maps: the configurations' FP16 rows, and the calibrated rows
+    (per head, and under one budget for all heads)."""
+    import torch
+
+    import quantized_linear_attention_damp_b200 as D
+    res = {}
+    for name in ("gdn_batch", "kda"):
+        w = W.WORKLOADS[name]
+        hs = W.head_structure(w)
+        acc = calibrate(w, dev)
+        cal_idx, _ = D.damp_calib_select(w.H, w.d, w.hp, acc)
+        is16_b, hp_b, _ = D.damp_calib_select_budget(w.H, w.d, w.hp * w.H, acc)
+        cal_map = np.zeros((w.H, w.d), np.uint8)
+        np.put_along_axis(cal_map, cal_idx.cpu().numpy().astype(np.int64), 1, axis=1)
+        pools = {"fp32": D.DampPool("fp32", w.n_slots, w.H, w.d, device=dev),
+                 "int8": D.DampPool("int8", w.n_slots, w.H, w.d, device=dev),
+                 "fp8": D.DampPool("fp8", w.n_slots, w.H, w.d, device=dev),
+                 "mixed_config_rows": D.DampPool("mixed", w.n_slots, w.H, w.d, hs.hp_row_idx,
+                                                 device=dev),
+                 "mixed_calibrated": D.DampPool("mixed", w.n_slots, w.H, w.d,
+                                                fp16_map=cal_map, device=dev),
+                 "mixed_calibrated_budget": D.DampPool("mixed", w.n_slots, w.H, w.d,
+                                                       fp16_map=is16_b.cpu().numpy(), device=dev)}
+        ident = torch.arange(w.n_slots, dtype=torch.int32, device=dev)
+        S0 = torch.from_numpy(W.initial_state(w, range(w.n_slots))).to(dev)
+        for p in pools.values():
+            p.pack(ident, S0)
+        out = torch.empty((w.n, w.H, w.d), dtype=torch.float32, device=dev)
+        cv = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        for s in range(steps):
+            x = W.step_inputs(w, s, hs)
+            t = [torch.from_numpy(x.slot_idx).to(dev), cv(x.q_bits), cv(x.k_bits), cv(x.v_bits),
+                 torch.from_numpy(x.alpha).to(dev), torch.from_numpy(x.beta).to(dev)]
+            for p in pools.values():
+                p.step(*t, out)
+        ref = torch.empty((w.n_slots, w.H, w.d, w.d), dtype=torch.float32, device=dev)
+        pools["fp32"].unpack(ident, ref)
+        cur = torch.empty_like(ref)
+        line = {"steps": steps, "fp16_rows_per_head_budget": w.hp,
+                "budget_rows_per_head_min_max": [int(hp_b.min()), int(hp_b.max())]}
+        for k, p in pools.items():
+            if k == "fp32":
+                continue
+            p.unpack(ident, cur)
+            line[k] = float(torch.linalg.vector_norm((cur - ref).double()) /
+                            torch.linalg.vector_norm(ref.double()))
+        for p in pools.values():
+            p.close()
+        res[name] = line
+    return res
+
+
+def serving(args, dev, steps: int = 16, warmup: int = 3):
+    """Context: the serving-shaped pool.  36 layer pools of 4096 slots x 32
+    heads (mixed format, d = 128; layers 3, 7, ... use KDA decay), one decode
+    step per layer per token on the same random 1024-slot subset.  Timed as
+    plain launches and as one CUDA graph replay per token.  Each layer's
+    q/k/v/alpha/beta are drawn once and reused; the slot subset changes every
+    step.  Needs about 97 GB of device memory; skipped (with the reason) if
+    that is not free."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import torch
+
+    import quantized_linear_attention_damp_b200 as D
+    from quantized_linear_attention_damp_b200.graph import DecodeGraph
+    L, nt = W.SERVING_LAYERS, W.SERVING_TEMPLATES
+    ws = [W.serving_layer(l) for l in range(L)]
+    pool_bytes = D.damp_pool_bytes(D.DAMP_FMT_MIXED, ws[0].n_slots, ws[0].H, ws[0].d, ws[0].d,
+                                   ws[0].hp)
+    free, _ = torch.cuda.mem_get_info(dev)
+    if free < L * pool_bytes + (8 << 30):
+        return {"skipped": f"needs {L * pool_bytes / 1e9:.1f} GB of pools, "
+                           f"{free / 1e9:.1f} GB free"}
+
+    def host(l):
+        hs = W.head_structure(ws[l])
+        return hs, W.serving_templates(ws[l]), W.serving_step_inputs(ws[l], 0, hs)
+
+    with ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+        gen = list(ex.map(host, range(L)))
+    pools, calls = [], []
+    slot_static = torch.empty(ws[0].n, dtype=torch.int32, device=dev)
+    for w, (hs, T, x) in zip(ws, gen):
+        p = D.DampPool("mixed", w.n_slots, w.H, w.d, hs.hp_row_idx, device=dev)
+        p.pack(torch.arange(nt, dtype=torch.int32, device=dev), torch.from_numpy(T).to(dev))
+        b = p.blocks()
+        g = w.n_slots // nt
+        b.view(g, nt, w.H, -1)[1:].copy_(b[:nt].unsqueeze(0).expand(g - 1, -1, -1, -1))
+        cv = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        a = dict(slot_idx=slot_static, q=cv(x.q_bits), k=cv(x.k_bits), v=cv(x.v_bits),
+                 alpha=torch.from_numpy(x.alpha).to(dev), beta=torch.from_numpy(x.beta).to(dev),
+                 out=torch.empty((w.n, w.H, w.d), dtype=torch.float32, device=dev))
+        pools.append(p)
+        calls.append((p, a))
+    del gen
+    n_total = warmup + steps
+    slot_tab = torch.from_numpy(np.stack([W.serving_slot_idx(s) for s in range(2 * n_total)]))
+    slot_tab = slot_tab.to(dev)
+    graph = DecodeGraph(calls, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def run(i, use_graph):
+        slot_static.copy_(slot_tab[i])
+        if use_graph:
+            graph.replay()
+        else:
+            for p, a in calls:
+                p.step(a["slot_idx"], a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["out"])
+
+    res = {"workload": f"serving pool: {L} layers x {ws[0].n_slots} slots x {ws[0].H} heads, "
+                       f"d_k=d_v={ws[0].d}, mixed state ({ws[0].hp} FP16 rows/head), "
+                       f"{ws[0].n} random slots per step, every 4th layer KDA, bf16 q/k/v",
+           "pool_bytes": L * pool_bytes}
+    step_bytes = sum(unit_bytes(w, "mixed") * w.n * w.H for w in ws)
+    units = sum(w.n * w.H for w in ws)
+    peak, _ = measured_peak()
+    for mode, use_graph in (("plain", False), ("graph", True)):
+        base = 0 if mode == "plain" else n_total
+        for i in range(warmup):
+            run(base + i, use_graph)
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            ev[i][0].record()
+            run(base + warmup + i, use_graph)
+            ev[i][1].record()
+        torch.cuda.synchronize(dev)
+        secs = sum(a_.elapsed_time(b_) for a_, b_ in ev) / 1e3
+        gbs = step_bytes * steps / secs / 1e9
+        res[mode] = {"ms_per_step": secs / steps * 1e3, "head_steps_per_s": units * steps / secs,
+                     "hbm_gbs": gbs, "frac": gbs / peak, "launches_per_step": L}
+    res["algorithmic_bytes_per_step"] = step_bytes
+    errs = [p.get_error() for p in pools]
+    res["error_flags"] = int(np.bitwise_or.reduce(errs))
+    graph.reset()
+    for p in pools:
+        p.close()
+    del calls, pools
+    torch.cuda.empty_cache()
     return res
 
 
@@ -436,9 +666,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="gdn_batch", choices=list(W.WORKLOADS))
-    ap.add_argument("--fmt", default="mixed", choices=["mixed", "int8", "fp32"])
+    ap.add_argument("--fmt", default="mixed", choices=["mixed", "int8", "fp8", "fp32"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-serving", action="store_true",
+                    help="skip the 36-layer serving-pool context run (about 97 GB)")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
