@@ -254,7 +254,8 @@ class Bench:
                 self.step(warmup + i)
                 ev[i][1].record()
             torch.cuda.synchronize(self.dev)
-        return sum(a.elapsed_time(b) for a, b in ev) / 1e3
+        self.step_ms = sorted(a.elapsed_time(b) for a, b in ev)
+        return sum(self.step_ms) / 1e3
 
     def timed_e2e(self, steps: int) -> tuple[float, int, int]:
         """Same steps through the public API from pinned host memory: each step
@@ -315,6 +316,17 @@ def cpu_baseline(w: W.Workload, fmt: str, seconds: float, max_units: int = 10 **
     return done / el, done, el
 
 
+def cpu_baseline_threads(w: W.Workload, fmt: str, seconds: float, threads: int):
+    """Oracle head-steps/s with `threads` host threads, each stepping its own
+    units (the same bounded sample per thread as cpu_baseline)."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(threads) as ex:
+        res = list(ex.map(lambda _: cpu_baseline(w, fmt, seconds), range(threads)))
+    n = sum(r[1] for r in res)
+    el = max(r[2] for r in res)
+    return n / el, n, el
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -359,6 +371,7 @@ def run_native(args, rank, world, local_rank):
                      "frac": gbs / peak, "peak_source": src,
                      "frac_of_8tbs_nominal": gbs / 8000.0,
                      "traffic": profiled_traffic(units)},
+        "step_us": {"median": b.step_ms[len(b.step_ms) // 2] * 1e3, "min": b.step_ms[0] * 1e3},
         "gpu_launches": args.steps,
         "clocks": sampler.summary(),
         "e2e": ({"value": units * world * args.steps / e2e_secs, "unit": "head-steps/s",
@@ -370,6 +383,12 @@ def run_native(args, rank, world, local_rank):
         line["cpu_baseline"] = {"value": v, "unit": "head-steps/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{n} (slot, head) units of {w.name} ({fmt}), "
                                           f"one step each, single thread, {el:.1f} s"}
+        t = os.cpu_count() or 1
+        v, n, el = cpu_baseline_threads(w, fmt, args.cpu_seconds, t)
+        line["cpu_baseline_all_cores"] = {
+            "value": v, "unit": "head-steps/s", "cores": t, "kind": "oracle",
+            "sample": f"{n} (slot, head) units of {w.name} ({fmt}), one step each, "
+                      f"{t} threads over units (the oracle's C calls release the GIL), {el:.1f} s"}
     if world == 1 and not args.no_variants:
         line["variants"] = variants(args, dev)
     if world == 1 and not args.no_variants:

@@ -17,8 +17,11 @@
 // tile in registers from dequantize to requantize.  u = k^T S' is summed in
 // the recursive pairwise order: 8 rows per thread as a subtree, then the top
 // four levels over the 16 row groups.  Warp 15, idle while columns are
-// combined, refills the pipeline (cp.async.bulk into a shared-memory ring of
-// stages completing on mbarriers, no tensor map, no multicast).
+// combined, writes back the previous item's blocks (one bulk store each, once
+// the barrier after phase A has ordered every writer's fenced rows before it)
+// and refills the pipeline (cp.async.bulk into a shared-memory ring of stages
+// completing on mbarriers, no tensor map, no multicast).  An item therefore
+// needs two CTA barriers, not three.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -62,8 +65,8 @@ __device__ __forceinline__ float bf16w(const uint32_t* w, int i) {
 
 // 8 INT8 codes (two words) times a scale, each product rounded once.
 __device__ __forceinline__ void dq_int8x8(uint2 w, float s, float2 (&x)[4]) {
-    dequant_int8x4_cvt(w.x, s, x[0], x[1]);
-    dequant_int8x4_cvt(w.y, s, x[2], x[3]);
+    dequant_int8x4_packed(w.x, s, x[0], x[1]);
+    dequant_int8x4_packed(w.y, s, x[2], x[3]);
 }
 __device__ __forceinline__ void dq_fp16x8(uint4 h, float2 (&x)[4]) {
     dequant_fp16x4(make_uint2(h.x, h.y), x[0], x[1]);
@@ -177,6 +180,18 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
             if (lane == 0)
                 bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)(uu % H) * kDirWords, kPD * 4, fb);
         }
+    };
+
+    // One bulk store per loaded block of item j (issue warp, lane 0).
+    auto store_item = [&](int j) {
+        const uint8_t* sj = smem + (size_t)(j % NS) * a.stage_bytes;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const PMeta m = *reinterpret_cast<const PMeta*>(sj + a.st_meta + w * sizeof(PMeta));
+            if (m.active == 1)
+                bulk_s2g(a.blocks + m.boff, smem_u32(sj + w * a.block_stride), m.bytes);
+        }
+        bulk_commit();
     };
 
     const int ahead = NS - 2;
@@ -300,14 +315,23 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
             for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
             if (cg == 0) cpart_s[ui * kPG + warp] = cp;
         }
-        if (tid == 0 && it >= 2) bulk_wait_read<1>();   // store of item it-2 has read its stage
         if (bar_red_or(0, kPT, ok ? 0 : 1)) {
             aborted = true;
             break;
         }
 
+        // ---- issue warp: write back item it-1 (its requantized rows were fenced by
+        // their writers before this barrier), then refill the stage of item it-2
+        // once that item's store has read it.
+        if (warp == kIssueWarp) {
+            if (lane == 0 && it >= 1) store_item(it - 1);
+            if (it + ahead < my_items) {
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+                issue(it + ahead);
+            }
+        }
         // ---- step 2 (second half) + step 3: delta_j and out_j, 2 x 128 columns
-        if (warp == kIssueWarp && it + ahead < my_items) issue(it + ahead);
         if (tid < 2 * kPD) {
             const int cu_ = tid >> 7, j = tid & (kPD - 1);
             const PMeta m = *reinterpret_cast<const PMeta*>(st + a.st_meta + cu_ * sizeof(PMeta));
@@ -401,27 +425,19 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
             }
             fence_proxy_async_smem();
         }
-        __syncthreads();
-
-        // ---- write back (one bulk store per block)
-        if (tid == 0) {
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-                const PMeta m = *reinterpret_cast<const PMeta*>(st + a.st_meta + w * sizeof(PMeta));
-                if (m.active == 1)
-                    bulk_s2g(a.blocks + m.boff, smem_u32(st + w * a.block_stride), m.bytes);
-            }
-            bulk_commit();
-        }
         if (++stage == NS) {
             stage = 0;
             parity ^= 1u;
         }
     }
 
-    if (tid == 0) {
+    // The last completed item (it-1) is still to be written back.
+    __syncthreads();
+    if (warp == kIssueWarp && lane == 0) {
+        if (it >= 1) store_item(it - 1);
         if (aborted) {
             atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
+            // drain loads that may still be landing in this CTA's stages
             for (int j = 0; j <= ahead; ++j) {
                 const int jt = it + j;
                 if (jt >= my_items) break;

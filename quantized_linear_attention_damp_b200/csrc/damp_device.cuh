@@ -337,10 +337,21 @@ __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off,
 // overlap.  Stores are made per the row's format.
 // ---------------------------------------------------------------------------
 
-// fl(code * scale) for 4 INT8 codes, converting each byte directly.
-__device__ __forceinline__ void dequant_int8x4_cvt(uint32_t w, float s, float2& lo, float2& hi) {
-    const float2 c01 = make_float2((float)(int8_t)(w & 0xffu), (float)(int8_t)((w >> 8) & 0xffu));
-    const float2 c23 = make_float2((float)(int8_t)((w >> 16) & 0xffu), (float)(int8_t)(w >> 24));
+// fl(code * scale) for 4 INT8 codes.  Each code, biased to 1..255, is placed
+// in the low mantissa bits of 2^23 by a byte permute; one exact packed
+// subtraction of 2^23 + 128 recovers the code and one packed multiply
+// applies the scale.  (Converting each byte with an integer-to-float
+// instruction measured ~5 % slower: those run on the quarter-rate
+// conversion pipe.)
+__device__ __forceinline__ void dequant_int8x4_packed(uint32_t w, float s, float2& lo, float2& hi) {
+    const uint32_t wb = w ^ 0x80808080u;
+    const float2 bias = f2(-8388736.0f);  // -(2^23 + 128)
+    float2 c01 = make_float2(__uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7440)),
+                             __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7441)));
+    float2 c23 = make_float2(__uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7442)),
+                             __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7443)));
+    c01 = __fadd2_rn(c01, bias);
+    c23 = __fadd2_rn(c23, bias);
     lo = __fmul2_rn(c01, f2(s));
     hi = __fmul2_rn(c23, f2(s));
 }
@@ -375,7 +386,7 @@ __device__ __forceinline__ void load_tile_dir(const uint8_t* blk, const uint32_t
         for (int j = 0; j < BATCH; ++j) {
             if (e[j] >> 31) dequant_fp16x4(w16[j], x[i0 + j][0], x[i0 + j][1]);
             else if constexpr (FP8) dequant_e4m3x4(w8[j], sc[j], x[i0 + j][0], x[i0 + j][1]);
-            else dequant_int8x4_cvt(w8[j], sc[j], x[i0 + j][0], x[i0 + j][1]);
+            else dequant_int8x4_packed(w8[j], sc[j], x[i0 + j][0], x[i0 + j][1]);
         }
     }
 }
