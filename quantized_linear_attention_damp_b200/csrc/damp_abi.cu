@@ -334,6 +334,7 @@ static int codec_args(const damp_pool* pool, int n, const int32_t* slot_idx, con
         return DAMP_ERR_MISALIGNED;
     a->blocks = d.dev_buf + d.header_bytes;
     a->masks = reinterpret_cast<const uint32_t*>(d.dev_buf + damp::kStatusBytes);
+    a->dir = reinterpret_cast<const uint32_t*>(d.dev_buf + d.dir_off);
     a->status = reinterpret_cast<uint32_t*>(d.dev_buf);
     a->slot_idx = slot_idx;
     a->state = const_cast<float*>(state);

@@ -157,22 +157,6 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
     return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
 }
 
-// Dequantize 4 INT8 codes (one 32-bit word) with an FP32 scale: fl(code*scale).
-// Codes are biased to 1..255 and placed in the mantissa of 2^23, so
-// (2^23 + c + 128) - (2^23 + 128) recovers c exactly without an I2F.
-__device__ __forceinline__ void dequant_int8x4(uint32_t w, float s, float2& lo, float2& hi) {
-    const uint32_t wb = w ^ 0x80808080u;
-    const float2 bias = f2(-8388736.0f);  // -(2^23 + 128)
-    float2 c01 = make_float2(__uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7440)),
-                             __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7441)));
-    float2 c23 = make_float2(__uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7442)),
-                             __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7443)));
-    c01 = __fadd2_rn(c01, bias);
-    c23 = __fadd2_rn(c23, bias);
-    lo = mul2_rn(c01, f2(s));
-    hi = mul2_rn(c23, f2(s));
-}
-
 __device__ __forceinline__ void dequant_fp16x4(uint2 h, float2& lo, float2& hi) {
     lo = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
     hi = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
@@ -255,32 +239,6 @@ __device__ __forceinline__ uint32_t quant_e4m3x4(float2 lo, float2 hi, float inv
     return (uint32_t)p01 | ((uint32_t)p23 << 16);
 }
 
-// Load rows [r0, r0+RPT) x cols [4cg, 4cg+4) of a quantized block into x
-// (dequantized, not decayed).
-template <int D, bool FP8 = false>
-__device__ __forceinline__ void load_quant_tile(const uint8_t* blk, uint32_t f16_off,
-                                                uint32_t i8_off, uint32_t bits, int rank16,
-                                                int r0, int cg, float2 (&x)[Geo<D>::RPT][2]) {
-    constexpr int RPT = Geo<D>::RPT;
-    int r16 = rank16, r8 = r0 - rank16;
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        if ((bits >> i) & 1u) {
-            const uint2 h =
-                *reinterpret_cast<const uint2*>(blk + f16_off + (size_t)r16 * (2 * D) + cg * 8);
-            dequant_fp16x4(h, x[i][0], x[i][1]);
-            ++r16;
-        } else {
-            const uint32_t w =
-                *reinterpret_cast<const uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4);
-            const float s = *reinterpret_cast<const float*>(blk + (size_t)r8 * 4);
-            if constexpr (FP8) dequant_e4m3x4(w, s, x[i][0], x[i][1]);
-            else dequant_int8x4(w, s, x[i][0], x[i][1]);
-            ++r8;
-        }
-    }
-}
-
 // Requantize rows [r0, r0+RPT) of x into a quantized block at `blk` (shared or
 // global).  rowbuf: 2*RPT floats private to this row group (shared memory).
 // Must be called by every lane of the warp (it synchronises the warp).
@@ -354,6 +312,36 @@ __device__ __forceinline__ void dequant_int8x4_packed(uint32_t w, float s, float
     c23 = __fadd2_rn(c23, bias);
     lo = __fmul2_rn(c01, f2(s));
     hi = __fmul2_rn(c23, f2(s));
+}
+
+// Rows [r0, r0+RPT) x cols [4cg, 4cg+4) of a quantized block in global memory,
+// addressed through the head's row directory.  Every row's loads are issued
+// before the first is used, so a thread's reads overlap instead of waiting one
+// after another behind the format branches.
+template <int D, bool FP8 = false>
+__device__ __forceinline__ void load_tile_gdir(const uint8_t* blk, const uint32_t* dir, int r0,
+                                               int cg, float2 (&x)[Geo<D>::RPT][2]) {
+    constexpr int RPT = Geo<D>::RPT;
+    uint32_t e[RPT];
+    uint2 raw[RPT];   // FP16 row: 4 values; byte row: 4 codes in .x, the row's scale in .y
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) e[i] = __ldg(dir + r0 + i);
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const uint8_t* row = blk + (e[i] & 0xffffu);
+        if (e[i] >> 31) {
+            raw[i] = __ldg(reinterpret_cast<const uint2*>(row + cg * 8));
+        } else {
+            raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(row + cg * 4));
+            raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(blk + ((e[i] >> 16) & 0x7fffu)));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        if (e[i] >> 31) dequant_fp16x4(raw[i], x[i][0], x[i][1]);
+        else if constexpr (FP8) dequant_e4m3x4(raw[i].x, __uint_as_float(raw[i].y), x[i][0], x[i][1]);
+        else dequant_int8x4_packed(raw[i].x, __uint_as_float(raw[i].y), x[i][0], x[i][1]);
+    }
 }
 
 // max(|a|, |b|, |c|, |d|) with a three-input maximum

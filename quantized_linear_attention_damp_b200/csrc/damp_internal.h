@@ -71,6 +71,7 @@ struct StepArgs {
 struct CodecArgs {
     uint8_t* blocks;
     const uint32_t* masks;
+    const uint32_t* dir;       // [H][128] row directory (quantized formats)
     uint32_t* status;
     const int32_t* slot_idx;
     float* state;              // [n][H][d][d]
