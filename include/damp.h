@@ -203,6 +203,17 @@ int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int 
                      const float* alpha, const float* beta, float* out, void* stream);
 
 /*
+ * Host-side check of a batch's slot indices (host int32 array [n]), for
+ * callers that want it before a step: every non-negative entry must be below
+ * n_slots and appear once.  Duplicates would give one block two writers in
+ * the same call (the in-place update of "STEPQuant ...", Appendix Table C2
+ * step 6, keeps one reader and one writer per block).  Returns DAMP_OK, or
+ * DAMP_ERR_INVALID_ARGUMENT with *bad_entry (may be NULL) set to the first
+ * offending batch position.  Reads host memory only; launches nothing.
+ */
+int damp_validate_slots(const int32_t* slot_idx, int n, int n_slots, int* bad_entry);
+
+/*
  * Read the device status word (DAMP_EFLAG_* bits accumulated since the last
  * clear) into *flags; clear it when `clear` is non-zero.  Synchronises
  * `stream`.

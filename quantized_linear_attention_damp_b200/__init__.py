@@ -53,7 +53,7 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing; build it with "
-            "`python -m quantized_linear_attention_damp_b200.build`")
+            "`python quantized_linear_attention_damp_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     sig = {
@@ -73,6 +73,7 @@ def _load():
         "damp_pool_create_map": (I, [I, I, I, I, P, P, S, ctypes.POINTER(P)]),
         "damp_pool_head_layout": (I, [P, I, ctypes.POINTER(S), ctypes.POINTER(S),
                                       ctypes.POINTER(S)]),
+        "damp_validate_slots": (I, [P, I, I, ctypes.POINTER(I)]),
         "damp_calib_bytes": (S, [I, I]),
         "damp_calib_accumulate": (I, [P, I, P, I, P, P, P]),
         "damp_calib_select": (I, [I, I, I, P, P, P, P]),
@@ -273,6 +274,18 @@ def damp_decode_step(pool: int, slot_idx: torch.Tensor, q: torch.Tensor, k: torc
                                  _stream(stream, q.device)), "damp_decode_step")
 
 
+def damp_validate_slots(slot_idx, n_slots: int) -> None:
+    """Host check of a batch's slot indices (distinct, below n_slots; negative
+    entries are padding).  Raises DampError naming the first bad entry."""
+    if isinstance(slot_idx, torch.Tensor):
+        slot_idx = slot_idx.detach().cpu().numpy()
+    s = np.ascontiguousarray(slot_idx, np.int32)
+    bad = ctypes.c_int(-1)
+    rc = _lib.damp_validate_slots(_ptr(s), s.size, n_slots, ctypes.byref(bad))
+    if rc != DAMP_OK:
+        raise DampError(rc, f"damp_validate_slots (entry {bad.value})")
+
+
 def damp_pool_get_error(pool: int, clear: bool = False, stream=None, device=None) -> int:
     f = ctypes.c_uint32()
     _check(_lib.damp_pool_get_error(pool, ctypes.byref(f), int(bool(clear)),
@@ -403,7 +416,11 @@ class DampPool:
     def unpack(self, slot_idx, state, stream=None):
         damp_pool_unpack(self.handle, slot_idx, state, stream)
 
-    def step(self, slot_idx, q, k, v, alpha, beta, out, stream=None):
+    def step(self, slot_idx, q, k, v, alpha, beta, out, stream=None, validate=False):
+        """One decode step; ``validate`` first checks the slot indices on the
+        host (a device-to-host copy: for debugging, not the serving path)."""
+        if validate:
+            damp_validate_slots(slot_idx, self.n_slots)
         damp_decode_step(self.handle, slot_idx, q, k, v, alpha, beta, out, stream)
 
     def get_error(self, clear=False, stream=None) -> int:

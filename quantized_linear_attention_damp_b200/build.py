@@ -1,6 +1,8 @@
 """Build libdamp.so (the CUDA library behind include/damp.h) for sm_100a, in-tree.
 
-    python -m quantized_linear_attention_damp_b200.build [--force]
+    python quantized_linear_attention_damp_b200/build.py [--force] [-v]
+
+(run as a file: importing the package itself needs the built library)
 
 Every translation unit is compiled with nvcc for sm_100a only, with
 -fmad=false (no implicit multiply-add contraction: the kernels spell out each

@@ -469,6 +469,22 @@ int damp_calib_select_budget(int H, int d_k, int budget, const double* acc, doub
                                                         static_cast<cudaStream_t>(stream)));
 }
 
+int damp_validate_slots(const int32_t* slot_idx, int n, int n_slots, int* bad_entry) {
+    if (bad_entry) *bad_entry = -1;
+    if (n < 0 || n_slots < 1 || (n > 0 && !slot_idx)) return DAMP_ERR_INVALID_ARGUMENT;
+    std::vector<uint8_t> seen((size_t)n_slots, 0);
+    for (int b = 0; b < n; ++b) {
+        const int32_t s = slot_idx[b];
+        if (s < 0) continue;
+        if (s >= n_slots || seen[(size_t)s]) {
+            if (bad_entry) *bad_entry = b;
+            return DAMP_ERR_INVALID_ARGUMENT;
+        }
+        seen[(size_t)s] = 1;
+    }
+    return DAMP_OK;
+}
+
 int damp_pool_get_error(const damp_pool* pool, uint32_t* flags, int clear, void* stream) {
     if (!pool || !flags || !pool->d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

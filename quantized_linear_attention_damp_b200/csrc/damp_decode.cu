@@ -9,16 +9,16 @@
 //   out = X^T q, before requantization                          step 3
 //   requantize X in place (FP16 rows, INT8 rows + FP32 scale)   step 6
 //
-// Work decomposition.  A persistent CTA of 9 warps walks work items (128/d
-// units each) with a grid stride.  Warp 8 is the producer: it reads the
-// per-unit metadata (slot, gates), waits until a shared-memory stage is free
-// and moves the unit's state block and inputs into it with cp.async.bulk
-// (no tensor map, no multicast), completing on the stage's "full" mbarrier.
-// Warps 0-7 consume: each thread keeps a (d/8) x 4 tile of the state in
-// registers from the dequantize through the requantize, so shared memory is
-// read once and written once per unit.  The new block is written back into
-// the same stage and thread 0 streams it to HBM with one bulk store, then
-// frees the stage one item later (after the store has read shared memory).
+// Work decomposition.  A persistent CTA of 8 warps walks work items (128/d
+// units each) with a grid stride.  Each thread keeps a (d/8) x 4 tile of the
+// state in registers from the dequantize through the requantize, so shared
+// memory is read once and written once per unit.  Warp 7, idle while columns
+// are combined, is also the issue warp: its lanes hold the next units'
+// metadata (slot, gates); it moves later units' state blocks and inputs into
+// free shared-memory stages with cp.async.bulk (no tensor map, no multicast),
+// completing on the stage's mbarrier.  Thread 0 writes each item's blocks
+// back with one bulk store each as soon as they are requantized; a stage is
+// refilled only after its store has read it.
 // The in-place update is safe because a unit's block has exactly one reader
 // and one writer per call (Table C2 step 6: the old representation stays
 // valid until its reader is done) -- slot indices within a call are distinct.
@@ -166,6 +166,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
     // Stage of item il is refilled with item il + NS - 2 at the start of
     // iteration il + ... : items il .. il + NS - 2 are in flight while item il
     // is consumed; the stage of item il - 1 is still being stored.
+    // One bulk store per loaded block of item j (thread 0).
+    auto store_item = [&](int j) {
+        const uint8_t* sj = smem + (size_t)(j % NS) * a.stage_bytes;
+        const int item_j = (int)blockIdx.x + j * (int)gridDim.x;
+#pragma unroll
+        for (int w = 0; w < UPI; ++w) {
+            const Meta m = *reinterpret_cast<const Meta*>(sj + a.st_meta + w * sizeof(Meta));
+            if (m.exists && m.slot >= 0 && m.slot < a.n_slots) {
+                const int uw = item_j * UPI + w;
+                const uint2 hb = __ldg(reinterpret_cast<const uint2*>(a.heads + uw % a.H));
+                bulk_s2g(a.blocks + (size_t)m.slot * a.slot_stride + hb.x,
+                         smem_u32(sj + w * a.block_stride), hb.y);
+            }
+        }
+        bulk_commit();
+    };
+
     const int ahead = NS - 2;
     if (warp == kIssueWarp)
         for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
@@ -337,21 +354,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             fence_proxy_async_smem();
         }
         __syncthreads();
-
-        // ---- write back (one bulk store per block)
-        if (tid == 0) {
-#pragma unroll
-            for (int w = 0; w < UPI; ++w) {
-                const Meta m = *reinterpret_cast<const Meta*>(st + a.st_meta + w * sizeof(Meta));
-                if (m.exists && m.slot >= 0 && m.slot < a.n_slots) {
-                    const int uw = item * UPI + w;
-                    const uint2 hb = __ldg(reinterpret_cast<const uint2*>(a.heads + uw % a.H));
-                    bulk_s2g(a.blocks + (size_t)m.slot * a.slot_stride + hb.x,
-                             smem_u32(st + w * a.block_stride), hb.y);
-                }
-            }
-            bulk_commit();
-        }
+        // ---- write back (one bulk store per block), right after the rows are
+        // written: with one CTA of large (FP32) blocks per SM and three stages,
+        // an earlier store frees the stage for the next load sooner
+        if (tid == 0) store_item(it);
     }
 
     if (tid == 0) {
@@ -523,17 +529,17 @@ cudaError_t prepare_decode(const PoolDesc& p) {
         case 64: return prepare_d<64>(c);
         case 128:
             if ((e = prepare_d<128>(c)) != cudaSuccess) return e;
-            return c == 1 ? prepare_decode_pair() : cudaSuccess;
+            return c != 0 ? prepare_decode_pair() : cudaSuccess;
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream) {
-    if (p.d == 128 && codec_of(p.format) == 1 && decode_pair_fits(a, in_dtype, gate)) {
+    if (p.d == 128 && codec_of(p.format) != 0 && decode_pair_fits(a, in_dtype, gate)) {
         StepArgs b = a;
         b.n_items = ((a.n + 1) / 2) * a.H;   // pairs of batch entries x heads
-        return launch_decode_pair(b, in_dtype, gate, stream);
+        return launch_decode_pair(b, in_dtype, gate, codec_of(p.format) == 2, stream);
     }
     switch (p.d) {
         case 16: return dispatch_fmt<16>(p, a, in_dtype, gate, stream);

@@ -64,9 +64,16 @@ __device__ __forceinline__ float bf16w(const uint32_t* w, int i) {
 }
 
 // 8 INT8 codes (two words) times a scale, each product rounded once.
-__device__ __forceinline__ void dq_int8x8(uint2 w, float s, float2 (&x)[4]) {
-    dequant_int8x4_packed(w.x, s, x[0], x[1]);
-    dequant_int8x4_packed(w.y, s, x[2], x[3]);
+// 8 byte-row codes (two words) times the row scale: INT8 or FP8 E4M3 codes.
+template <bool FP8>
+__device__ __forceinline__ void dq_byte8(uint2 w, float s, float2 (&x)[4]) {
+    if constexpr (FP8) {
+        dequant_e4m3x4(w.x, s, x[0], x[1]);
+        dequant_e4m3x4(w.y, s, x[2], x[3]);
+    } else {
+        dequant_int8x4_packed(w.x, s, x[0], x[1]);
+        dequant_int8x4_packed(w.y, s, x[2], x[3]);
+    }
 }
 __device__ __forceinline__ void dq_fp16x8(uint4 h, float2 (&x)[4]) {
     dequant_fp16x4(make_uint2(h.x, h.y), x[0], x[1]);
@@ -81,7 +88,7 @@ __device__ __forceinline__ float absmax8(const float2 (&x)[4]) {
     return fmaxf(m, fabsf(x[3].y));
 }
 
-template <bool KDA, bool BF16>
+template <bool KDA, bool BF16, bool FP8>
 __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     constexpr uint32_t ELT = BF16 ? 2 : 4;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     if (dir[i0 + j] >> 31) dq_fp16x8(w16[j], x[i0 + j]);
-                    else dq_int8x8(w8[j], sc[j], x[i0 + j]);
+                    else dq_byte8<FP8>(w8[j], sc[j], x[i0 + j]);
                 }
             }
             // ---- step 2 (first half): S' = D S^; u = k^T S' (pairwise); w = q^T S'
@@ -394,7 +401,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 const uint32_t e = sdir[cg];
                 if (!(e >> 31)) {
                     float scale, inv;
-                    row_scale(rowbuf[cg], scale, inv);
+                    row_scale<FP8>(rowbuf[cg], scale, inv);
                     rowbuf[kPR + cg] = inv;
                     *reinterpret_cast<float*>(blk + ((e >> 16) & 0x7fffu)) = scale;
                 }
@@ -419,8 +426,10 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                         make_uint4(h0.x, h0.y, h1.x, h1.y);
                 } else {
                     *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + off) =
-                        make_uint2(quant_int8x4(x[i][0], x[i][1], inv[i]),
-                                   quant_int8x4(x[i][2], x[i][3], inv[i]));
+                        FP8 ? make_uint2(quant_e4m3x4(x[i][0], x[i][1], inv[i]),
+                                         quant_e4m3x4(x[i][2], x[i][3], inv[i]))
+                            : make_uint2(quant_int8x4(x[i][0], x[i][1], inv[i]),
+                                         quant_int8x4(x[i][2], x[i][3], inv[i]));
                 }
             }
             fence_proxy_async_smem();
@@ -480,21 +489,21 @@ uint32_t pair_layout(StepArgs& a, bool kda, bool bf16) {
     return ns;
 }
 
-template <bool KDA, bool BF16>
+template <bool KDA, bool BF16, bool FP8>
 cudaError_t pair_attrs_t() {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(decode_pair_kernel<KDA, BF16>,
+        attr_err = cudaFuncSetAttribute(decode_pair_kernel<KDA, BF16, FP8>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     });
     return attr_err;
 }
 
-template <bool KDA, bool BF16>
+template <bool KDA, bool BF16, bool FP8>
 cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
-    auto kern = decode_pair_kernel<KDA, BF16>;
-    const cudaError_t attr_err = pair_attrs_t<KDA, BF16>();
+    auto kern = decode_pair_kernel<KDA, BF16, FP8>;
+    const cudaError_t attr_err = pair_attrs_t<KDA, BF16, FP8>();
     if (attr_err != cudaSuccess) return attr_err;
     StepArgs a = a0;
     int dev = 0, sms = 0;
@@ -514,10 +523,14 @@ cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
 
 cudaError_t prepare_decode_pair() {
     cudaError_t e;
-    if ((e = pair_attrs_t<false, false>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<false, true>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<true, false>()) != cudaSuccess) return e;
-    return pair_attrs_t<true, true>();
+    if ((e = pair_attrs_t<false, false, false>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<false, true, false>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<true, false, false>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<true, true, false>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<false, false, true>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<false, true, true>()) != cudaSuccess) return e;
+    if ((e = pair_attrs_t<true, false, true>()) != cudaSuccess) return e;
+    return pair_attrs_t<true, true, true>();
 }
 
 bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate) {
@@ -525,10 +538,18 @@ bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate) {
     return pair_layout(b, gate == DAMP_GATE_VECTOR, in_dtype == DAMP_DTYPE_BF16) != 0;
 }
 
-cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, cudaStream_t stream) {
+cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, bool fp8,
+                               cudaStream_t stream) {
     const bool kda = gate == DAMP_GATE_VECTOR, bf = in_dtype == DAMP_DTYPE_BF16;
-    if (kda) return bf ? launch_pair_t<true, true>(a, stream) : launch_pair_t<true, false>(a, stream);
-    return bf ? launch_pair_t<false, true>(a, stream) : launch_pair_t<false, false>(a, stream);
+    if (fp8) {
+        if (kda)
+            return bf ? launch_pair_t<true, true, true>(a, stream)
+                      : launch_pair_t<true, false, true>(a, stream);
+        return bf ? launch_pair_t<false, true, true>(a, stream)
+                  : launch_pair_t<false, false, true>(a, stream);
+    }
+    if (kda) return bf ? launch_pair_t<true, true, false>(a, stream) : launch_pair_t<true, false, false>(a, stream);
+    return bf ? launch_pair_t<false, true, false>(a, stream) : launch_pair_t<false, false, false>(a, stream);
 }
 
 }  // namespace damp

@@ -96,7 +96,8 @@ cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtyp
                                cudaStream_t stream);
 // d = 128 quantized states, two units of one head per CTA iteration
 // (damp_decode_pair.cu); a.n_items counts pairs x heads.
-cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, cudaStream_t stream);
+cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, bool fp8,
+                               cudaStream_t stream);
 bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate);   // >= 3 stages fit
 // One-time kernel attribute set-up for every decode variant a pool can launch
 // (called by damp_pool_create, outside any stream capture).

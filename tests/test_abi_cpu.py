@@ -220,3 +220,12 @@ def test_per_head_map_layout():
         bad = same.copy()
         bad[0, 0] = 2
         D.damp_pool_bytes_map(5, H, d, d, bad)
+
+
+def test_validate_slots():
+    D.damp_validate_slots(np.array([3, -1, 0, 5, -1], np.int32), 6)
+    D.damp_validate_slots(np.zeros(0, np.int32), 1)
+    for bad, pos in ((np.array([1, 2, 1], np.int32), 2), (np.array([0, 6], np.int32), 1)):
+        with pytest.raises(D.DampError) as ei:
+            D.damp_validate_slots(bad, 6)
+        assert ei.value.status == D.DAMP_ERR_INVALID_ARGUMENT and f"entry {pos}" in str(ei.value)

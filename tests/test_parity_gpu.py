@@ -196,6 +196,31 @@ def test_identity_step_keeps_codes_on_gpu():
         p.close()
 
 
+def test_delta_rule_write_invariant_on_gpu():
+    """FP32 state, unit k (normalised in FP32 inputs), beta = alpha = 1: the
+    step writes v along k, so k^T X = v^T to 1e-5 (relative to the state's
+    size) for every unit of the batch."""
+    w = W.Workload("inv_fp32", n=6, n_slots=8, H=4, d=128, hp=0, steps=1, gate=W.GATE_GDN,
+                   in_dtype="f32")
+    p = Pair(w, "fp32", oracle_slots=[0])
+    try:
+        x = W.step_inputs(w, 0, p.hs)
+        k64 = x.k.astype(np.float64)
+        x.k = (k64 / np.linalg.norm(k64, axis=-1, keepdims=True)).astype(np.float32)
+        x.alpha[:] = 1.0
+        x.beta[:] = 1.0
+        S0 = p.gpu.read_logical()["f32"]
+        p.gpu_step(x)
+        X = p.gpu.read_logical()["f32"].astype(np.float64)
+        for b, slot in enumerate(x.slot_idx):
+            for h in range(w.H):
+                kx = x.k[b, h].astype(np.float64) @ X[slot, h]
+                bound = 1e-5 * max(1.0, float(np.abs(S0[slot, h]).max()))
+                assert np.abs(kx - x.v[b, h]).max() <= bound, (b, h)
+    finally:
+        p.close()
+
+
 def test_unpack_matches_oracle_reconstruction():
     w = SMALL["d64_kda_bf16"]
     p = Pair(w, "mixed")
