@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <mutex>
 
 #include "damp.h"
@@ -111,44 +112,65 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     // ---- issue side (warp 15): lane L holds the metadata of CTA-local unit
     // U == L (mod 32), loaded 32 units ahead of use.
     constexpr int kIssueWarp = kPT / 32 - 1;
+    // The ring holds raw values: the loads are issued here and nothing waits
+    // for them until the unit is issued, 16 items later (a branch on the
+    // freshly loaded slot index used to stall the issue warp on every refill).
+    struct RMeta {
+        int slot;          // slot index; INT_MIN: no such batch entry
+        float alpha, beta;
+        int unit;
+        int head;
+        uint2 hb;          // the head's {block offset in the slot, block size}
+    };
     auto load_meta = [&](int U) {
-        PMeta m{0, 0u, 0.f, 0.f, -1, -1};
+        RMeta r{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
         if (U < my_units) {
             const int g = (int)blockIdx.x + (U >> 1) * (int)gridDim.x;  // item: pair p, head h
             const int p = g / H, h = g - p * H;
             const int b = 2 * p + (U & 1);
+            r.head = h;
             if (b < a.n) {
-                const long long u = (long long)b * H + h;
-                const int slot = __ldg(a.slot_idx + b);
-                m.unit = u;
-                if constexpr (!KDA) m.alpha = __ldg(a.alpha + u);
-                m.beta = __ldg(a.beta + u);
-                if (slot >= 0 && slot < a.n_slots) {
-                    const uint2 hb = __ldg(reinterpret_cast<const uint2*>(a.heads + h));
-                    m.active = 1;
-                    m.bytes = hb.y;
-                    m.boff = (long long)slot * (long long)a.slot_stride + hb.x;
-                } else if (slot >= a.n_slots) {
-                    m.active = -1;   // out of range: flagged by the consumer
-                }
+                const int u = b * H + h;
+                r.slot = __ldg(a.slot_idx + b);
+                r.unit = u;
+                if constexpr (!KDA) r.alpha = __ldg(a.alpha + u);
+                r.beta = __ldg(a.beta + u);
+                r.hb = __ldg(reinterpret_cast<const uint2*>(a.heads + h));
+            }
+        }
+        return r;
+    };
+    // Stage metadata of a unit from its raw ring values.
+    auto finish_meta = [&](const RMeta& r) {
+        PMeta m{0, 0u, r.alpha, r.beta, -1, -1};
+        if (r.slot != INT_MIN) {
+            m.unit = r.unit;
+            if (r.slot >= 0 && r.slot < a.n_slots) {
+                m.active = 1;
+                m.bytes = r.hb.y;
+                m.boff = (long long)r.slot * (long long)a.slot_stride + r.hb.x;
+            } else if (r.slot >= a.n_slots) {
+                m.active = -1;   // out of range: flagged by the consumer
             }
         }
         return m;
     };
-    PMeta ring{0, 0u, 0.f, 0.f, -1, -1};
+    RMeta ring{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
     if (warp == kIssueWarp) ring = load_meta(lane);
 
     auto issue = [&](int il) {
         const int stage = il % NS;
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
         const int src = (2 * il + lane) & 31;
-        PMeta m;
-        m.active = __shfl_sync(0xffffffffu, ring.active, src);
-        m.bytes = __shfl_sync(0xffffffffu, ring.bytes, src);
-        m.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
-        m.beta = __shfl_sync(0xffffffffu, ring.beta, src);
-        m.unit = __shfl_sync(0xffffffffu, ring.unit, src);
-        m.boff = __shfl_sync(0xffffffffu, ring.boff, src);
+        RMeta r;
+        r.slot = __shfl_sync(0xffffffffu, ring.slot, src);
+        r.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
+        r.beta = __shfl_sync(0xffffffffu, ring.beta, src);
+        r.unit = __shfl_sync(0xffffffffu, ring.unit, src);
+        r.head = __shfl_sync(0xffffffffu, ring.head, src);
+        r.hb.x = __shfl_sync(0xffffffffu, ring.hb.x, src);
+        r.hb.y = __shfl_sync(0xffffffffu, ring.hb.y, src);
+        const PMeta m = finish_meta(r);
         const int rel = (lane - 2 * il) & 31;
         if (rel < 2) ring = load_meta(2 * il + rel + 32);
         const bool load = lane < 2 && m.active == 1;
@@ -180,13 +202,8 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 bulk_g2s(smem_u32(st + a.st_alpha + lane * kPD * 4), a.alpha + (size_t)m.unit * kPD,
                          kPD * 4, fb);
         }
-        if (loads) {
-            // both units of the item share head h = unit mod H
-            const int hl = __ffs(loads) - 1;
-            const long long uu = __shfl_sync(0xffffffffu, m.unit, hl);
-            if (lane == 0)
-                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)(uu % H) * kDirWords, kPD * 4, fb);
-        }
+        if (loads && lane == 0)   // both units of the item share head h
+            bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirWords, kPD * 4, fb);
     };
 
     // One bulk store per loaded block of item j (issue warp, lane 0).
@@ -365,9 +382,9 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 const float vj = in_at<BF16>(st + a.st_v + cu_ * kPD * ELT, j);
                 const float dj = __fsub_rn(vj, uj);
                 delta_s[cu_ * kPD + j] = dj;
-                a.out[m.unit * kPD + j] = __fmaf_rn(c, dj, wj);
+                a.out[(size_t)m.unit * kPD + j] = __fmaf_rn(c, dj, wj);
             } else if (m.unit >= 0) {
-                a.out[m.unit * kPD + j] = 0.f;
+                a.out[(size_t)m.unit * kPD + j] = 0.f;
                 if (j == 0 && m.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
             }
         }
