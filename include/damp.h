@@ -72,6 +72,7 @@ extern "C" {
 #define DAMP_ERR_MISALIGNED (-3)       /* a pointer is not 16-byte aligned      */
 #define DAMP_ERR_BUFFER_TOO_SMALL (-4) /* buf_bytes < damp_pool_bytes(...)      */
 #define DAMP_ERR_CUDA (-5)             /* a CUDA runtime call failed            */
+#define DAMP_ERR_TIMEOUT (-6)          /* a host wait on the stream hit its limit */
 
 /* ---- device status word bits (damp_pool_get_error) ----------------------- */
 #define DAMP_EFLAG_SLOT_RANGE 1u /* a slot_idx entry >= n_slots (entry skipped) */
@@ -215,8 +216,9 @@ int damp_validate_slots(const int32_t* slot_idx, int n, int n_slots, int* bad_en
 
 /*
  * Read the device status word (DAMP_EFLAG_* bits accumulated since the last
- * clear) into *flags; clear it when `clear` is non-zero.  Synchronises
- * `stream`.
+ * clear) into *flags; clear it when `clear` is non-zero.  Waits for the work
+ * already queued on `stream` by polling, for at most 10 s: DAMP_ERR_TIMEOUT
+ * (nothing read, nothing cleared) if it has not finished by then.
  */
 int damp_pool_get_error(const damp_pool* pool, uint32_t* flags, int clear, void* stream);
 

@@ -26,6 +26,7 @@ DAMP_ERR_UNSUPPORTED = -2
 DAMP_ERR_MISALIGNED = -3
 DAMP_ERR_BUFFER_TOO_SMALL = -4
 DAMP_ERR_CUDA = -5
+DAMP_ERR_TIMEOUT = -6
 
 DAMP_EFLAG_SLOT_RANGE = 1
 DAMP_EFLAG_TIMEOUT = 2

@@ -7,7 +7,9 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <chrono>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "damp.h"
@@ -74,6 +76,7 @@ const char* damp_status_string(int status) {
         case DAMP_ERR_MISALIGNED: return "pointer not 16-byte aligned";
         case DAMP_ERR_BUFFER_TOO_SMALL: return "pool buffer too small";
         case DAMP_ERR_CUDA: return "CUDA runtime error";
+        case DAMP_ERR_TIMEOUT: return "host wait on the stream timed out";
         default: return "unknown status";
     }
 }
@@ -488,11 +491,33 @@ int damp_validate_slots(const int32_t* slot_idx, int n, int n_slots, int* bad_en
 int damp_pool_get_error(const damp_pool* pool, uint32_t* flags, int clear, void* stream) {
     if (!pool || !flags || !pool->d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Wait for the work already queued by polling an event, with a deadline,
+    // so that a stream that never drains is reported instead of waited on.
+    cudaEvent_t ev;
+    cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return DAMP_ERR_CUDA;
+    e = cudaEventRecord(ev, s);
+    const auto deadline = std::chrono::steady_clock::now() + std::chrono::seconds(10);
+    while (e == cudaSuccess) {
+        const cudaError_t q = cudaEventQuery(ev);
+        if (q == cudaSuccess) break;
+        if (q != cudaErrorNotReady) {
+            e = q;
+            break;
+        }
+        if (std::chrono::steady_clock::now() > deadline) {
+            cudaEventDestroy(ev);
+            return DAMP_ERR_TIMEOUT;
+        }
+        std::this_thread::sleep_for(std::chrono::microseconds(50));
+    }
+    cudaEventDestroy(ev);
+    if (e != cudaSuccess) return DAMP_ERR_CUDA;
     uint32_t* st = reinterpret_cast<uint32_t*>(pool->d.dev_buf);
     uint32_t host = 0;
-    cudaError_t e = cudaMemcpyAsync(&host, st, 4, cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(&host, st, 4, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess && clear) e = cudaMemsetAsync(st, 0, 4, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);   // the two tiny operations above
     if (e != cudaSuccess) return DAMP_ERR_CUDA;
     *flags = host;
     return DAMP_OK;

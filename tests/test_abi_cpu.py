@@ -103,7 +103,7 @@ def test_layout_rejects_bad_shapes(args, status):
 
 
 def test_status_strings():
-    for s in (0, -1, -2, -3, -4, -5, -99):
+    for s in (0, -1, -2, -3, -4, -5, -6, -99):
         assert isinstance(D.damp_status_string(s), str) and D.damp_status_string(s)
 
 
