@@ -16,12 +16,13 @@
 // 0-15 work on unit 0, lanes 16-31 on unit 1.  Each thread keeps its 8 x 8
 // tile in registers from dequantize to requantize.  u = k^T S' is summed in
 // the recursive pairwise order: 8 rows per thread as a subtree, then the top
-// four levels over the 16 row groups.  Warp 15, idle while columns are
-// combined, writes back the previous item's blocks (one bulk store each, once
-// the barrier after phase A has ordered every writer's fenced rows before it)
-// and refills the pipeline (cp.async.bulk into a shared-memory ring of stages
-// completing on mbarriers, no tensor map, no multicast).  An item therefore
-// needs two CTA barriers, not three.
+// four levels over the 16 row groups.  While columns are combined, warp 14
+// writes back the previous item's blocks (one bulk store each, once the
+// barrier after phase A has ordered every writer's fenced rows before it) and
+// warp 15 refills the pipeline (cp.async.bulk into a shared-memory ring of
+// stages completing on mbarriers, no tensor map, no multicast); a named
+// barrier between the two lets the refill start as soon as the stage's old
+// store has read it.  An item needs two CTA barriers, not three.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -347,13 +348,17 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         // ---- issue warp: write back item it-1 (its requantized rows were fenced by
         // their writers before this barrier), then refill the stage of item it-2
         // once that item's store has read it.
-        if (warp == kIssueWarp) {
+        // warp kIssueWarp-1 writes back; kIssueWarp refills.  The store warp
+        // first checks that the store of item it-2 has read its stage (the
+        // stage refilled below), releases the issue warp, then stores item it-1.
+        if (warp == kIssueWarp - 1) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            asm volatile("bar.arrive 2, 64;" ::: "memory");
             if (lane == 0 && it >= 1) store_item(it - 1);
-            if (it + ahead < my_items) {
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-                issue(it + ahead);
-            }
+        } else if (warp == kIssueWarp) {
+            asm volatile("bar.sync 2, 64;" ::: "memory");
+            if (it + ahead < my_items) issue(it + ahead);
         }
         // ---- step 2 (second half) + step 3: delta_j and out_j, 2 x 128 columns
         if (tid < 2 * kPD) {
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
 
     // The last completed item (it-1) is still to be written back.
     __syncthreads();
-    if (warp == kIssueWarp && lane == 0) {
+    if (warp == kIssueWarp - 1 && lane == 0) {
         if (it >= 1) store_item(it - 1);
         if (aborted) {
             atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
