@@ -19,10 +19,13 @@
 // four levels over the 16 row groups.  While columns are combined, warp 14
 // writes back the previous item's blocks (one bulk store each, once the
 // barrier after phase A has ordered every writer's fenced rows before it) and
-// warp 15 refills the pipeline (cp.async.bulk into a shared-memory ring of
-// stages completing on mbarriers, no tensor map, no multicast); a named
-// barrier between the two lets the refill start as soon as the stage's old
-// store has read it.  An item needs two CTA barriers, not three.
+// warps 15 and 13 refill the pipeline (cp.async.bulk into a shared-memory ring
+// of stages completing on mbarriers, no tensor map, no multicast): warp 15
+// the metadata, the two blocks and the row directory, warp 13 q, k, v (and
+// the KDA decays), each arriving once on the stage's mbarrier with its own
+// byte count.  A named barrier among the three lets the refill start as soon
+// as the stage's old store has read it.  An item needs two CTA barriers, not
+// three.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 1);
+        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 2);   // two refill warps
         fence_mbar_init();
     }
     __syncthreads();
@@ -110,9 +113,12 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     const int my_items = (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int my_units = 2 * my_items;
 
-    // ---- issue side (warp 15): lane L holds the metadata of CTA-local unit
-    // U == L (mod 32), loaded 32 units ahead of use.
+    // ---- issue side (warps 15 and 13): lane L holds the metadata of CTA-local
+    // unit U == L (mod 32), loaded 32 units ahead of use; both refill warps
+    // keep the same ring.
     constexpr int kIssueWarp = kPT / 32 - 1;
+    constexpr int kInputWarp = kIssueWarp - 2;   // q, k, v (and alpha) copies
+    const bool refill = warp == kIssueWarp || warp == kInputWarp;
     // The ring holds raw values: the loads are issued here and nothing waits
     // for them until the unit is issued, 16 items later (a branch on the
     // freshly loaded slot index used to stall the issue warp on every refill).
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         return m;
     };
     RMeta ring{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
-    if (warp == kIssueWarp) ring = load_meta(lane);
+    if (refill) ring = load_meta(lane);
 
     auto issue = [&](int il) {
         const int stage = il % NS;
@@ -176,11 +182,16 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         if (rel < 2) ring = load_meta(2 * il + rel + 32);
         const bool load = lane < 2 && m.active == 1;
         const uint32_t loads = __ballot_sync(0xffffffffu, load);
+        const bool lead = warp == kIssueWarp;   // metadata, blocks, directory
         uint32_t tx = 0;
         if (lane < 2) {
-            *reinterpret_cast<PMeta*>(st + a.st_meta + lane * sizeof(PMeta)) = m;
-            if (load) tx = m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u);
-            if (lane == 0 && loads) tx += 4u * kPD;   // the head's row directory
+            if (lead) {
+                *reinterpret_cast<PMeta*>(st + a.st_meta + lane * sizeof(PMeta)) = m;
+                if (load) tx = m.bytes;
+                if (lane == 0 && loads) tx += 4u * kPD;   // the head's row directory
+            } else if (load) {
+                tx = 3u * kPD * ELT + (KDA ? 4u * kPD : 0u);
+            }
         }
         const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
         __syncwarp();
@@ -190,8 +201,11 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         }
         __syncwarp();
         const uint32_t fb = full_bar(stage);
-        if (load) {
-            bulk_g2s(smem_u32(st + lane * a.block_stride), a.blocks + m.boff, m.bytes, fb);
+        if (lead) {
+            if (load) bulk_g2s(smem_u32(st + lane * a.block_stride), a.blocks + m.boff, m.bytes, fb);
+            if (loads && lane == 0)   // both units of the item share head h
+                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirWords, kPD * 4, fb);
+        } else if (load) {
             const size_t io = (size_t)m.unit * kPD * ELT;
             bulk_g2s(smem_u32(st + a.st_q + lane * kPD * ELT),
                      static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
@@ -203,8 +217,6 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 bulk_g2s(smem_u32(st + a.st_alpha + lane * kPD * 4), a.alpha + (size_t)m.unit * kPD,
                          kPD * 4, fb);
         }
-        if (loads && lane == 0)   // both units of the item share head h
-            bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirWords, kPD * 4, fb);
     };
 
     // One bulk store per loaded block of item j (issue warp, lane 0).
@@ -220,7 +232,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     };
 
     const int ahead = NS - 2;
-    if (warp == kIssueWarp)
+    if (refill)
         for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
 
     // ---- consumers
@@ -345,19 +357,18 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
             break;
         }
 
-        // ---- issue warp: write back item it-1 (its requantized rows were fenced by
-        // their writers before this barrier), then refill the stage of item it-2
-        // once that item's store has read it.
-        // warp kIssueWarp-1 writes back; kIssueWarp refills.  The store warp
-        // first checks that the store of item it-2 has read its stage (the
-        // stage refilled below), releases the issue warp, then stores item it-1.
+        // ---- write back item it-1 (its requantized rows were fenced by their
+        // writers before this barrier) and refill the stage of item it-2 once
+        // that item's store has read it.  The store warp (kIssueWarp-1) first
+        // checks that the store of item it-2 has read its stage, releases the
+        // two refill warps through named barrier 2, then stores item it-1.
         if (warp == kIssueWarp - 1) {
             if (lane == 0) bulk_wait_read<0>();
             __syncwarp();
-            asm volatile("bar.arrive 2, 64;" ::: "memory");
+            asm volatile("bar.arrive 2, 96;" ::: "memory");
             if (lane == 0 && it >= 1) store_item(it - 1);
-        } else if (warp == kIssueWarp) {
-            asm volatile("bar.sync 2, 64;" ::: "memory");
+        } else if (refill) {
+            asm volatile("bar.sync 2, 96;" ::: "memory");
             if (it + ahead < my_items) issue(it + ahead);
         }
         // ---- step 2 (second half) + step 3: delta_j and out_j, 2 x 128 columns
