@@ -39,8 +39,8 @@ import workloads as W  # noqa: E402
 
 METRIC = "head-steps/s and achieved HBM GB/s (% of B200 roofline) per decode step"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["damp_decode_pair.cu", "damp_device.cuh", "damp_internal.h"]   # the profiled kernel
-PROFILE = os.path.join(ROOT, "profiles", "decode_pair_hiconc_gdn_mixed.txt")
+KERNEL_SOURCES = ["damp_decode_unit.cu", "damp_device.cuh", "damp_internal.h"]   # the profiled kernel
+PROFILE = os.path.join(ROOT, "profiles", "decode_unit_hiconc_gdn_mixed.txt")
 
 
 # ---------------------------------------------------------------- accounting

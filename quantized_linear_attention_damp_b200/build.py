@@ -22,7 +22,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdamp.so")
-SOURCES = ["damp_abi.cu", "damp_decode.cu", "damp_decode_pair.cu", "damp_codec.cu",
+SOURCES = ["damp_abi.cu", "damp_decode.cu", "damp_decode_unit.cu", "damp_codec.cu",
            "damp_calib.cu"]
 HEADERS = ["damp_internal.h", "damp_device.cuh"]
 

@@ -529,17 +529,17 @@ cudaError_t prepare_decode(const PoolDesc& p) {
         case 64: return prepare_d<64>(c);
         case 128:
             if ((e = prepare_d<128>(c)) != cudaSuccess) return e;
-            return c != 0 ? prepare_decode_pair() : cudaSuccess;
+            return c != 0 ? prepare_decode_unit() : cudaSuccess;
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream) {
-    if (p.d == 128 && codec_of(p.format) != 0 && decode_pair_fits(a, in_dtype, gate)) {
+    if (p.d == 128 && codec_of(p.format) != 0 && decode_unit_fits(a, in_dtype, gate)) {
         StepArgs b = a;
-        b.n_items = ((a.n + 1) / 2) * a.H;   // pairs of batch entries x heads
-        return launch_decode_pair(b, in_dtype, gate, codec_of(p.format) == 2, stream);
+        b.n_items = a.n * a.H;   // units
+        return launch_decode_unit(b, in_dtype, gate, codec_of(p.format) == 2, stream);
     }
     switch (p.d) {
         case 16: return dispatch_fmt<16>(p, a, in_dtype, gate, stream);

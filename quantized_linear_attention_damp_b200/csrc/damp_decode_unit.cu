@@ -1,31 +1,31 @@
-// damp_decode_pair.cu -- decode step for quantized d = 128 states, two units
-// of the same head per CTA iteration.
+// damp_decode_unit.cu -- decode step for quantized d = 128 states, one unit
+// (slot, head) per CTA iteration, two CTAs per SM.
 //
 // Same arithmetic, same order of operations and same results as the generic
 // kernel in damp_decode.cu ("STEPQuant ...", Appendix Table C2 steps 1, 2,
 // 3, 6 on the DAMP row format); only the work decomposition differs.
 //
-// Why pairs.  A lane owns 8 columns of a row, so one row of one unit takes 16
-// lanes and a warp covers the same row of two units.  The two units are the
-// same head h of two batch entries, so they share the head's FP16-row map
-// and every row is FP16 or INT8 for the whole warp: format branches stay
-// warp-uniform while the per-row work (directory lookup, scale, k/q values,
-// row maximum, division, stores) is spread over 8 columns instead of 4.
+// CTA of 8 warps.  Half-warp hh of warp w owns key rows [8g, 8g + 8) of the
+// unit, g = 2w + hh; a lane owns 8 columns, so one row takes 16 lanes.  Each
+// thread keeps its 8 x 8 tile in registers from dequantize to requantize, and
+// the per-row work (directory lookup, scale, k/q values, row maximum,
+// division, stores) is spread over 8 columns.  The two halves of a warp work
+// on different rows, so a format branch runs both paths, each for its half,
+// when the rows differ in format.  u = k^T S' is summed in the recursive
+// pairwise order: 8 rows per thread as a subtree, then the top four levels
+// over the 16 row groups.
 //
-// CTA of 16 warps: warp w owns key rows [8w, 8w + 8) of both units; lanes
-// 0-15 work on unit 0, lanes 16-31 on unit 1.  Each thread keeps its 8 x 8
-// tile in registers from dequantize to requantize.  u = k^T S' is summed in
-// the recursive pairwise order: 8 rows per thread as a subtree, then the top
-// four levels over the 16 row groups.  While columns are combined, warp 14
-// writes back the previous item's blocks (one bulk store each, once the
-// barrier after phase A has ordered every writer's fenced rows before it) and
-// warps 15 and 13 refill the pipeline (cp.async.bulk into a shared-memory ring
-// of stages completing on mbarriers, no tensor map, no multicast): warp 15
-// the metadata, the two blocks and the row directory, warp 13 q, k, v (and
-// the KDA decays), each arriving once on the stage's mbarrier with its own
-// byte count.  A named barrier among the three lets the refill start as soon
-// as the stage's old store has read it.  An item needs two CTA barriers, not
-// three.
+// Two CTAs share an SM whenever three stages fit in half of its shared
+// memory (4 stages at 27 FP16 rows): their barriers are independent, so one CTA's arithmetic fills the
+// other's barrier waits.  While columns are combined, warp 6 writes back the
+// previous unit's block (one bulk store, once the barrier after phase A has
+// ordered every writer's fenced rows before it) and warp 7 refills the
+// pipeline (cp.async.bulk of the block, q, k, v, the KDA decays and the
+// head's row directory into a shared-memory ring of stages completing on
+// mbarriers; no tensor map, no multicast).  A named barrier between the two
+// lets the refill start as soon as the stage's old store has read it.  An
+// item needs two CTA barriers, not three.
+
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -38,12 +38,12 @@
 namespace damp {
 namespace {
 
-constexpr int kPT = 512;       // threads
+constexpr int kPT = 256;       // threads (8 warps)
 constexpr int kPD = 128;       // d_k = d_v
 constexpr int kPR = 8;         // rows per thread
-constexpr int kPG = 16;        // row groups (warps)
+constexpr int kPG = 16;        // row groups (half-warps)
 
-// Per-unit metadata written by the issue warp into the stage (32 bytes).
+// Per-unit metadata written by the refill warp into the stage (32 bytes).
 struct PMeta {
     int active;        // 1: block loaded, to be updated and stored
     uint32_t bytes;    // block size of the unit's head
@@ -68,7 +68,6 @@ __device__ __forceinline__ float bf16w(const uint32_t* w, int i) {
     return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
 }
 
-// 8 INT8 codes (two words) times a scale, each product rounded once.
 // 8 byte-row codes (two words) times the row scale: INT8 or FP8 E4M3 codes.
 template <bool FP8>
 __device__ __forceinline__ void dq_byte8(uint2 w, float s, float2 (&x)[4]) {
@@ -94,7 +93,7 @@ __device__ __forceinline__ float absmax8(const float2 (&x)[4]) {
 }
 
 template <bool KDA, bool BF16, bool FP8>
-__global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
+__global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     constexpr uint32_t ELT = BF16 ? 2 : 4;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
@@ -104,26 +103,22 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 2);   // two refill warps
+        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 1);
         fence_mbar_init();
     }
     __syncthreads();
 
     const int H = a.H;
     const int my_items = (a.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int my_units = 2 * my_items;
 
-    // ---- issue side (warps 15 and 13): lane L holds the metadata of CTA-local
-    // unit U == L (mod 32), loaded 32 units ahead of use; both refill warps
-    // keep the same ring.
-    constexpr int kIssueWarp = kPT / 32 - 1;
-    constexpr int kInputWarp = kIssueWarp - 2;   // q, k, v (and alpha) copies
-    const bool refill = warp == kIssueWarp || warp == kInputWarp;
-    // The ring holds raw values: the loads are issued here and nothing waits
-    // for them until the unit is issued, 16 items later (a branch on the
-    // freshly loaded slot index used to stall the issue warp on every refill).
+    // ---- refill side (warp 7): lane L holds the metadata of CTA-local unit
+    // U == L (mod 32), loaded 32 units ahead of use.  The ring holds raw
+    // values: nothing waits for the loads until the unit is issued, and no
+    // branch depends on a freshly loaded slot index.
+    constexpr int kIssueWarp = kPT / 32 - 1;    // refill
+    constexpr int kStoreWarp = kIssueWarp - 1;  // write-back
     struct RMeta {
-        int slot;          // slot index; INT_MIN: no such batch entry
+        int slot;          // slot index; INT_MIN: no such unit
         float alpha, beta;
         int unit;
         int head;
@@ -131,19 +126,15 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     };
     auto load_meta = [&](int U) {
         RMeta r{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
-        if (U < my_units) {
-            const int g = (int)blockIdx.x + (U >> 1) * (int)gridDim.x;  // item: pair p, head h
-            const int p = g / H, h = g - p * H;
-            const int b = 2 * p + (U & 1);
+        if (U < my_items) {
+            const int u = (int)blockIdx.x + U * (int)gridDim.x;   // unit b*H + h
+            const int b = u / H, h = u - b * H;
             r.head = h;
-            if (b < a.n) {
-                const int u = b * H + h;
-                r.slot = __ldg(a.slot_idx + b);
-                r.unit = u;
-                if constexpr (!KDA) r.alpha = __ldg(a.alpha + u);
-                r.beta = __ldg(a.beta + u);
-                r.hb = __ldg(reinterpret_cast<const uint2*>(a.heads + h));
-            }
+            r.slot = __ldg(a.slot_idx + b);
+            r.unit = u;
+            if constexpr (!KDA) r.alpha = __ldg(a.alpha + u);
+            r.beta = __ldg(a.beta + u);
+            r.hb = __ldg(reinterpret_cast<const uint2*>(a.heads + h));
         }
         return r;
     };
@@ -163,12 +154,14 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         return m;
     };
     RMeta ring{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
-    if (refill) ring = load_meta(lane);
+    if (warp == kIssueWarp) ring = load_meta(lane);
 
+    // Refill the stage of item il: metadata, then one bulk copy per operand,
+    // all completing on the stage's mbarrier (lane 0 issues them).
     auto issue = [&](int il) {
         const int stage = il % NS;
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
-        const int src = (2 * il + lane) & 31;
+        const int src = il & 31;
         RMeta r;
         r.slot = __shfl_sync(0xffffffffu, ring.slot, src);
         r.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
@@ -178,74 +171,51 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
         r.hb.x = __shfl_sync(0xffffffffu, ring.hb.x, src);
         r.hb.y = __shfl_sync(0xffffffffu, ring.hb.y, src);
         const PMeta m = finish_meta(r);
-        const int rel = (lane - 2 * il) & 31;
-        if (rel < 2) ring = load_meta(2 * il + rel + 32);
-        const bool load = lane < 2 && m.active == 1;
-        const uint32_t loads = __ballot_sync(0xffffffffu, load);
-        const bool lead = warp == kIssueWarp;   // metadata, blocks, directory
-        uint32_t tx = 0;
-        if (lane < 2) {
-            if (lead) {
-                *reinterpret_cast<PMeta*>(st + a.st_meta + lane * sizeof(PMeta)) = m;
-                if (load) tx = m.bytes;
-                if (lane == 0 && loads) tx += 4u * kPD;   // the head's row directory
-            } else if (load) {
-                tx = 3u * kPD * ELT + (KDA ? 4u * kPD : 0u);
+        if (lane == src) ring = load_meta(il + 32);
+        if (lane == 0) {
+            *reinterpret_cast<PMeta*>(st + a.st_meta) = m;
+            const uint32_t fb = full_bar(stage);
+            if (m.active == 1) {
+                mbar_arrive_expect_tx(fb, m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u) + 4u * kPD);
+                bulk_g2s(smem_u32(st), a.blocks + m.boff, m.bytes, fb);
+                const size_t io = (size_t)m.unit * kPD * ELT;
+                bulk_g2s(smem_u32(st + a.st_q), static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
+                bulk_g2s(smem_u32(st + a.st_k), static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
+                bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
+                if constexpr (KDA)
+                    bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + (size_t)m.unit * kPD, kPD * 4, fb);
+                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirWords, kPD * 4, fb);
+            } else {
+                mbar_arrive(fb);
             }
         }
-        const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
         __syncwarp();
-        if (lane == 0) {
-            if (tx_all) mbar_arrive_expect_tx(full_bar(stage), tx_all);
-            else mbar_arrive(full_bar(stage));
-        }
-        __syncwarp();
-        const uint32_t fb = full_bar(stage);
-        if (lead) {
-            if (load) bulk_g2s(smem_u32(st + lane * a.block_stride), a.blocks + m.boff, m.bytes, fb);
-            if (loads && lane == 0)   // both units of the item share head h
-                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirWords, kPD * 4, fb);
-        } else if (load) {
-            const size_t io = (size_t)m.unit * kPD * ELT;
-            bulk_g2s(smem_u32(st + a.st_q + lane * kPD * ELT),
-                     static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
-            bulk_g2s(smem_u32(st + a.st_k + lane * kPD * ELT),
-                     static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
-            bulk_g2s(smem_u32(st + a.st_v + lane * kPD * ELT),
-                     static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
-            if constexpr (KDA)
-                bulk_g2s(smem_u32(st + a.st_alpha + lane * kPD * 4), a.alpha + (size_t)m.unit * kPD,
-                         kPD * 4, fb);
-        }
     };
 
-    // One bulk store per loaded block of item j (issue warp, lane 0).
+    // One bulk store of item j's block (store warp, lane 0).
     auto store_item = [&](int j) {
         const uint8_t* sj = smem + (size_t)(j % NS) * a.stage_bytes;
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            const PMeta m = *reinterpret_cast<const PMeta*>(sj + a.st_meta + w * sizeof(PMeta));
-            if (m.active == 1)
-                bulk_s2g(a.blocks + m.boff, smem_u32(sj + w * a.block_stride), m.bytes);
-        }
+        const PMeta m = *reinterpret_cast<const PMeta*>(sj + a.st_meta);
+        if (m.active == 1) bulk_s2g(a.blocks + m.boff, smem_u32(sj), m.bytes);
         bulk_commit();
     };
 
     const int ahead = NS - 2;
-    if (refill)
+    if (warp == kIssueWarp)
         for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
 
-    // ---- consumers
-    const int ui = lane >> 4;           // unit of the pair
+    // ---- consumers: half-warp hh of warp w owns row group 2w + hh
+    const int hh = lane >> 4;
     const int cg = lane & 15;           // columns 8cg .. 8cg+7
-    const int r0 = warp * kPR;          // rows r0 .. r0+7
+    const int rg = warp * 2 + hh;       // row group
+    const int r0 = rg * kPR;            // rows r0 .. r0+7
 
     uint8_t* scratch = smem + a.scratch_off;
-    float* red_u = reinterpret_cast<float*>(scratch);            // [2][16][128]
-    float* red_w = red_u + 2 * kPG * kPD;                        // [2][16][128]
-    float* delta_s = red_w + 2 * kPG * kPD;                      // [2][128]
-    float* cpart_s = delta_s + 2 * kPD;                          // [2][16]
-    float* rowbuf = cpart_s + 2 * kPG + (warp * 2 + ui) * 16;    // this half-warp's 16 floats
+    float* red_u = reinterpret_cast<float*>(scratch);   // [16][128]
+    float* red_w = red_u + kPG * kPD;                   // [16][128]
+    float* delta_s = red_w + kPG * kPD;                 // [128]
+    float* cpart_s = delta_s + kPD;                     // [16]
+    float* rowbuf = cpart_s + kPG + rg * 16;            // this half-warp's 16 floats
 
     int it = 0, stage = 0;
     uint32_t parity = 0;
@@ -253,27 +223,23 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     for (; it < my_items; ++it) {
         const bool ok = mbar_wait_bounded(full_bar(stage), parity);
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
-        const PMeta meta = *reinterpret_cast<const PMeta*>(st + a.st_meta + ui * sizeof(PMeta));
-        const PMeta mo = *reinterpret_cast<const PMeta*>(st + a.st_meta + (ui ^ 1) * sizeof(PMeta));
-        // The directory (and so every row offset) is valid only if at least one
-        // unit of the item was loaded; this is uniform over the CTA.
-        const bool any = ok && (meta.active == 1 || mo.active == 1);
-        uint8_t* blk = st + ui * a.block_stride;
-        const uint8_t* sq = st + a.st_q + ui * kPD * ELT;
-        const uint8_t* sk = st + a.st_k + ui * kPD * ELT;
-        const float* salpha = reinterpret_cast<const float*>(st + a.st_alpha) + ui * kPD;
+        const PMeta meta = *reinterpret_cast<const PMeta*>(st + a.st_meta);
+        const bool any = ok && meta.active == 1;
+        uint8_t* blk = st;
+        const uint8_t* sq = st + a.st_q;
+        const uint8_t* sk = st + a.st_k;
+        const float* salpha = reinterpret_cast<const float*>(st + a.st_alpha);
         const uint32_t* sdir = reinterpret_cast<const uint32_t*>(st + a.st_dir) + r0;
-        const uint8_t* b16 = blk + cg * 16;   // this lane's 16 bytes of an FP16 row
-        const uint8_t* b8 = blk + cg * 8;     // this lane's 8 bytes of an INT8 row
+        const uint8_t* b16 = blk + cg * 16;
+        const uint8_t* b8 = blk + cg * 8;
 
-        // Every lane computes (an inactive half works on stale stage data
-        // and skips every global side effect), so warp-level operations
-        // always see a full warp.
         float2 x[kPR][4];
         uint32_t kw[BF16 ? kPR / 2 : 1], qw[BF16 ? kPR / 2 : 1];
         auto kval = [&](int i) { return BF16 ? bf16w(kw, i) : in_at<false>(sk, r0 + i); };
         auto qval = [&](int i) { return BF16 ? bf16w(qw, i) : in_at<false>(sq, r0 + i); };
         uint32_t dir[kPR];
+        // `any` is uniform over the CTA: the directory (and so every row
+        // offset) is valid only for a loaded unit.
         if (any) {
             if constexpr (BF16) {
                 const uint4 kv = *reinterpret_cast<const uint4*>(sk + 2 * r0);
@@ -338,8 +304,8 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                     for (int c = 0; c < 4; ++c) us[c] = v[c];
                 }
             }
-            float* ru = red_u + (ui * kPG + warp) * kPD + 8 * cg;
-            float* rw = red_w + (ui * kPG + warp) * kPD + 8 * cg;
+            float* ru = red_u + rg * kPD + 8 * cg;
+            float* rw = red_w + rg * kPD + 8 * cg;
             reinterpret_cast<float4*>(ru)[0] = make_float4(us[0].x, us[0].y, us[1].x, us[1].y);
             reinterpret_cast<float4*>(ru)[1] = make_float4(us[2].x, us[2].y, us[3].x, us[3].y);
             reinterpret_cast<float4*>(rw)[0] = make_float4(ws[0].x, ws[0].y, ws[1].x, ws[1].y);
@@ -350,7 +316,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                                          __fmul_rn(meta.beta, in_at<BF16>(sk, r0 + cg)));
 #pragma unroll
             for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
-            if (cg == 0) cpart_s[ui * kPG + warp] = cp;
+            if (cg == 0) cpart_s[rg] = cp;
         }
         if (bar_red_or(0, kPT, ok ? 0 : 1)) {
             aborted = true;
@@ -359,24 +325,22 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
 
         // ---- write back item it-1 (its requantized rows were fenced by their
         // writers before this barrier) and refill the stage of item it-2 once
-        // that item's store has read it.  The store warp (kIssueWarp-1) first
-        // checks that the store of item it-2 has read its stage, releases the
-        // two refill warps through named barrier 2, then stores item it-1.
-        if (warp == kIssueWarp - 1) {
+        // that item's store has read it: the store warp checks the read,
+        // releases the refill warp through named barrier 2, then stores.
+        if (warp == kStoreWarp) {
             if (lane == 0) bulk_wait_read<0>();
             __syncwarp();
-            asm volatile("bar.arrive 2, 96;" ::: "memory");
+            asm volatile("bar.arrive 2, 64;" ::: "memory");
             if (lane == 0 && it >= 1) store_item(it - 1);
-        } else if (refill) {
-            asm volatile("bar.sync 2, 96;" ::: "memory");
+        } else if (warp == kIssueWarp) {
+            asm volatile("bar.sync 2, 64;" ::: "memory");
             if (it + ahead < my_items) issue(it + ahead);
         }
-        // ---- step 2 (second half) + step 3: delta_j and out_j, 2 x 128 columns
-        if (tid < 2 * kPD) {
-            const int cu_ = tid >> 7, j = tid & (kPD - 1);
-            const PMeta m = *reinterpret_cast<const PMeta*>(st + a.st_meta + cu_ * sizeof(PMeta));
-            if (m.active == 1) {
-                const float* c0 = red_u + cu_ * kPG * kPD + j;
+        // ---- step 2 (second half) + step 3: delta_j and out_j, 128 columns
+        if (tid < kPD) {
+            const int j = tid;
+            if (meta.active == 1) {
+                const float* c0 = red_u + j;
                 float t[8];
 #pragma unroll
                 for (int q2 = 0; q2 < 8; ++q2)
@@ -384,31 +348,31 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 const float uj = __fadd_rn(
                     __fadd_rn(__fadd_rn(t[0], t[1]), __fadd_rn(t[2], t[3])),
                     __fadd_rn(__fadd_rn(t[4], t[5]), __fadd_rn(t[6], t[7])));
-                const float* w0 = red_w + cu_ * kPG * kPD + j;
+                const float* w0 = red_w + j;
                 float wj = 0.f;
 #pragma unroll
                 for (int q2 = 0; q2 < kPG; ++q2) wj = __fadd_rn(wj, w0[q2 * kPD]);
-                const float4* cpp = reinterpret_cast<const float4*>(cpart_s + cu_ * kPG);
+                const float4* cpp = reinterpret_cast<const float4*>(cpart_s);
                 float c = 0.f;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const float4 v4 = cpp[q4];
                     c += (v4.x + v4.y) + (v4.z + v4.w);
                 }
-                const float vj = in_at<BF16>(st + a.st_v + cu_ * kPD * ELT, j);
+                const float vj = in_at<BF16>(st + a.st_v, j);
                 const float dj = __fsub_rn(vj, uj);
-                delta_s[cu_ * kPD + j] = dj;
-                a.out[(size_t)m.unit * kPD + j] = __fmaf_rn(c, dj, wj);
-            } else if (m.unit >= 0) {
-                a.out[(size_t)m.unit * kPD + j] = 0.f;
-                if (j == 0 && m.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
+                delta_s[j] = dj;
+                a.out[(size_t)meta.unit * kPD + j] = __fmaf_rn(c, dj, wj);
+            } else if (meta.unit >= 0) {
+                a.out[(size_t)meta.unit * kPD + j] = 0.f;
+                if (j == 0 && meta.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
             }
         }
         __syncthreads();
 
         // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
         if (any) {
-            const float4* dp = reinterpret_cast<const float4*>(delta_s + ui * kPD + 8 * cg);
+            const float4* dp = reinterpret_cast<const float4*>(delta_s + 8 * cg);
             const float4 d0 = dp[0], d1 = dp[1];
             const float2 dl[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
                                   make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
@@ -418,12 +382,12 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
                 const float b = __fmul_rn(meta.beta, kval(i));
 #pragma unroll
                 for (int c = 0; c < 4; ++c) x[i][c] = __ffma2_rn(f2(b), dl[c], x[i][c]);
-                // row maxima of both units with full-warp reductions (the other
-                // half contributes 0, the smallest |x|)
+                // row maxima of both half-warps with full-warp reductions (the
+                // other half contributes 0, the smallest |x|)
                 const uint32_t mb = __float_as_uint(absmax8(x[i]));
-                const uint32_t m0 = __reduce_max_sync(0xffffffffu, ui ? 0u : mb);
-                const uint32_t m1 = __reduce_max_sync(0xffffffffu, ui ? mb : 0u);
-                amax[i] = __uint_as_float(ui ? m1 : m0);
+                const uint32_t m0 = __reduce_max_sync(0xffffffffu, hh ? 0u : mb);
+                const uint32_t m1 = __reduce_max_sync(0xffffffffu, hh ? mb : 0u);
+                amax[i] = __uint_as_float(hh ? m1 : m0);
             }
             if (cg == 0) {
                 reinterpret_cast<float4*>(rowbuf)[0] = make_float4(amax[0], amax[1], amax[2], amax[3]);
@@ -475,7 +439,7 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
 
     // The last completed item (it-1) is still to be written back.
     __syncthreads();
-    if (warp == kIssueWarp - 1 && lane == 0) {
+    if (warp == kStoreWarp && lane == 0) {
         if (it >= 1) store_item(it - 1);
         if (aborted) {
             atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
@@ -491,28 +455,27 @@ __global__ void __launch_bounds__(kPT, 1) decode_pair_kernel(const StepArgs a) {
     }
 }
 
-// Stage layout of the pair kernel; returns the number of stages that fit
-// (0 when fewer than three do).
-uint32_t pair_layout(StepArgs& a, bool kda, bool bf16) {
+// Stage layout within `budget` bytes of shared memory; returns the number of
+// stages that fit (0 when fewer than three do).
+uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
     const uint32_t elt = bf16 ? 2 : 4;
     auto up = [](uint32_t x, uint32_t m) { return (x + m - 1) / m * m; };
-    uint32_t off = 2 * a.block_stride;
+    uint32_t off = a.block_stride;
     a.st_q = off;
-    off = up(off + 2 * kPD * elt, 16);
+    off = up(off + kPD * elt, 16);
     a.st_k = off;
-    off = up(off + 2 * kPD * elt, 16);
+    off = up(off + kPD * elt, 16);
     a.st_v = off;
-    off = up(off + 2 * kPD * elt, 16);
+    off = up(off + kPD * elt, 16);
     a.st_alpha = off;
-    off += kda ? 2 * kPD * 4 : 0;
+    off += kda ? kPD * 4 : 0;
     a.st_mask = off;
     a.st_dir = off;
     off += kPD * 4;
     a.st_meta = off;
-    off += 2 * sizeof(PMeta);
+    off += sizeof(PMeta);
     a.stage_bytes = up(off, 128);
-    const uint32_t scratch = up((2 * 2 * kPG * kPD + 2 * kPD + 2 * kPG + kPG * 2 * 16) * 4, 128);
-    const uint32_t budget = 227u * 1024u;
+    const uint32_t scratch = up((2 * kPG * kPD + kPD + kPG + kPG * 16) * 4, 128);
     uint32_t ns = (budget - scratch - 128) / a.stage_bytes;
     if (ns > 6) ns = 6;
     if (ns < 3) return 0;
@@ -522,21 +485,29 @@ uint32_t pair_layout(StepArgs& a, bool kda, bool bf16) {
     return ns;
 }
 
+// Shared memory of one CTA: 227 KB alone on an SM; two CTAs share the SM's
+// 228 KB, less 1 KB reserved per CTA.
+constexpr uint32_t kBudget1 = 227u * 1024u;
+constexpr uint32_t kBudget2 = 228u * 1024u / 2 - 1024u;
+
 template <bool KDA, bool BF16, bool FP8>
-cudaError_t pair_attrs_t() {
+cudaError_t unit_attrs_t() {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(decode_pair_kernel<KDA, BF16, FP8>,
+        attr_err = cudaFuncSetAttribute(decode_unit_kernel<KDA, BF16, FP8>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode_unit_kernel<KDA, BF16, FP8>,
+                                            cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     });
     return attr_err;
 }
 
 template <bool KDA, bool BF16, bool FP8>
-cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
-    auto kern = decode_pair_kernel<KDA, BF16, FP8>;
-    const cudaError_t attr_err = pair_attrs_t<KDA, BF16, FP8>();
+cudaError_t launch_unit_t(const StepArgs& a0, cudaStream_t stream) {
+    auto kern = decode_unit_kernel<KDA, BF16, FP8>;
+    const cudaError_t attr_err = unit_attrs_t<KDA, BF16, FP8>();
     if (attr_err != cudaSuccess) return attr_err;
     StepArgs a = a0;
     int dev = 0, sms = 0;
@@ -544,45 +515,52 @@ cudaError_t launch_pair_t(const StepArgs& a0, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    const uint32_t ns = pair_layout(a, KDA, BF16);
+    // two CTAs per SM when 3 stages fit in half of it, else one CTA
+    uint32_t ns = unit_layout(a, KDA, BF16, kBudget2);
+    if (ns == 0) ns = unit_layout(a, KDA, BF16, kBudget1);
     if (ns == 0) return cudaErrorInvalidConfiguration;
     const size_t smem = a.bar_off + 8u * ns;
-    const int grid = std::min(a.n_items, sms);
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPT, smem)) != cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int grid = std::min(a.n_items, sms * per_sm);
+    if (grid <= 0) return cudaSuccess;
     kern<<<grid, kPT, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t prepare_decode_pair() {
+cudaError_t prepare_decode_unit() {
     cudaError_t e;
-    if ((e = pair_attrs_t<false, false, false>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<false, true, false>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<true, false, false>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<true, true, false>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<false, false, true>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<false, true, true>()) != cudaSuccess) return e;
-    if ((e = pair_attrs_t<true, false, true>()) != cudaSuccess) return e;
-    return pair_attrs_t<true, true, true>();
+    if ((e = unit_attrs_t<false, false, false>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<false, true, false>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<true, false, false>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<true, true, false>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<false, false, true>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<false, true, true>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<true, false, true>()) != cudaSuccess) return e;
+    return unit_attrs_t<true, true, true>();
 }
 
-bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate) {
+bool decode_unit_fits(const StepArgs& a, int in_dtype, int gate) {
     StepArgs b = a;
-    return pair_layout(b, gate == DAMP_GATE_VECTOR, in_dtype == DAMP_DTYPE_BF16) != 0;
+    return unit_layout(b, gate == DAMP_GATE_VECTOR, in_dtype == DAMP_DTYPE_BF16, kBudget1) != 0;
 }
 
-cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, bool fp8,
+cudaError_t launch_decode_unit(const StepArgs& a, int in_dtype, int gate, bool fp8,
                                cudaStream_t stream) {
     const bool kda = gate == DAMP_GATE_VECTOR, bf = in_dtype == DAMP_DTYPE_BF16;
     if (fp8) {
         if (kda)
-            return bf ? launch_pair_t<true, true, true>(a, stream)
-                      : launch_pair_t<true, false, true>(a, stream);
-        return bf ? launch_pair_t<false, true, true>(a, stream)
-                  : launch_pair_t<false, false, true>(a, stream);
+            return bf ? launch_unit_t<true, true, true>(a, stream)
+                      : launch_unit_t<true, false, true>(a, stream);
+        return bf ? launch_unit_t<false, true, true>(a, stream)
+                  : launch_unit_t<false, false, true>(a, stream);
     }
-    if (kda) return bf ? launch_pair_t<true, true, false>(a, stream) : launch_pair_t<true, false, false>(a, stream);
-    return bf ? launch_pair_t<false, true, false>(a, stream) : launch_pair_t<false, false, false>(a, stream);
+    if (kda) return bf ? launch_unit_t<true, true, false>(a, stream) : launch_unit_t<true, false, false>(a, stream);
+    return bf ? launch_unit_t<false, true, false>(a, stream) : launch_unit_t<false, false, false>(a, stream);
 }
 
 }  // namespace damp

@@ -94,15 +94,15 @@ struct CalibArgs {
 // Launchers (damp_decode.cu, damp_codec.cu, damp_calib.cu).  They return cudaError_t.
 cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
                                cudaStream_t stream);
-// d = 128 quantized states, two units of one head per CTA iteration
-// (damp_decode_pair.cu); a.n_items counts pairs x heads.
-cudaError_t launch_decode_pair(const StepArgs& a, int in_dtype, int gate, bool fp8,
+// d = 128 quantized states, one unit per CTA iteration, two CTAs per SM
+// (damp_decode_unit.cu); a.n_items counts units (n x H).
+cudaError_t launch_decode_unit(const StepArgs& a, int in_dtype, int gate, bool fp8,
                                cudaStream_t stream);
-bool decode_pair_fits(const StepArgs& a, int in_dtype, int gate);   // >= 3 stages fit
+bool decode_unit_fits(const StepArgs& a, int in_dtype, int gate);   // >= 3 stages fit
 // One-time kernel attribute set-up for every decode variant a pool can launch
 // (called by damp_pool_create, outside any stream capture).
 cudaError_t prepare_decode(const PoolDesc& p);
-cudaError_t prepare_decode_pair();
+cudaError_t prepare_decode_unit();
 cudaError_t launch_calib_accumulate(const CalibArgs& a, int d, cudaStream_t stream);
 cudaError_t launch_calib_select(const double* acc, int H, int d, int hp, double* score,
                                 uint16_t* idx, cudaStream_t stream);

@@ -100,8 +100,8 @@ def test_per_head_fp16_row_counts(name):
     run_full(w, "mixed", min(w.steps, 4), fp16_map=random_map(w.H, w.d, counts, w.H * w.d))
 
 
-def test_per_head_fp16_row_counts_pair_kernel():
-    """d = 128 with every head's block small enough for the two-unit kernel's
+def test_per_head_fp16_row_counts_unit_kernel():
+    """d = 128 with every head's block small enough for the d = 128 kernel's
     stages (no all-FP16 head)."""
     w = SMALL["d128_ragged"].with_(name="d128_varhp", H=6)
     counts = [0, 27, 60, 1, 100, 27]
