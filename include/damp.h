@@ -115,8 +115,8 @@ int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
 
 /*
  * Bytes the caller must allocate for a pool of n_slots x H blocks: a header
- * (device status word, per-head FP16-row masks, row directory and block
- * table, 256 B aligned) followed by the slots.  With one FP16-row count for
+ * (device status word, per-head FP16-row masks, row directory with the
+ * row-group order, and block table, 256 B aligned) followed by the slots.  With one FP16-row count for
  * every head, block (slot, h) is at header + (slot*H + h)*stride.
  */
 int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
@@ -158,6 +158,18 @@ int damp_pool_create_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is
  * Any output pointer may be NULL. */
 int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,
                           size_t* block_stride, size_t* offset_in_slot);
+
+/*
+ * Head h's row-group order, as the d = 128 decode step uses it (a work
+ * decomposition only: results do not depend on it).  The kernel gives each
+ * half-warp one group of 8 consecutive key rows, two groups per warp; a warp
+ * whose two groups differ in format at a row position runs both format paths
+ * there.  order[16] (host) receives the groups g (rows 8g .. 8g+7) in
+ * half-warp order, paired so that the number of such positions over the
+ * head is the minimum over all pairings (exact; ties to the lower group).
+ * The pool header stores the same order after the head's row directory.
+ */
+int damp_pool_row_groups(const damp_pool* pool, int h, uint8_t* order);
 
 /* Release the descriptor (never the caller's device buffer).  NULL is a no-op. */
 int damp_pool_destroy(damp_pool* pool);

@@ -74,6 +74,7 @@ def _load():
         "damp_pool_create_map": (I, [I, I, I, I, P, P, S, ctypes.POINTER(P)]),
         "damp_pool_head_layout": (I, [P, I, ctypes.POINTER(S), ctypes.POINTER(S),
                                       ctypes.POINTER(S)]),
+        "damp_pool_row_groups": (I, [P, I, P]),
         "damp_validate_slots": (I, [P, I, I, ctypes.POINTER(I)]),
         "damp_calib_bytes": (S, [I, I]),
         "damp_calib_accumulate": (I, [P, I, P, I, P, P, P]),
@@ -195,6 +196,14 @@ def damp_pool_head_layout(pool: int, h: int) -> tuple[int, int, int]:
     _check(_lib.damp_pool_head_layout(pool, h, ctypes.byref(b), ctypes.byref(s),
                                       ctypes.byref(o)), "damp_pool_head_layout")
     return b.value, s.value, o.value
+
+
+def damp_pool_row_groups(pool: int, h: int) -> list[int]:
+    """Head h's row-group order: the group (key rows 8g .. 8g+7) of each
+    half-warp of the d = 128 decode step, two per warp."""
+    order = (ctypes.c_uint8 * 16)()
+    _check(_lib.damp_pool_row_groups(pool, h, order), "damp_pool_row_groups")
+    return list(order)
 
 
 def damp_pool_destroy(pool: int) -> None:

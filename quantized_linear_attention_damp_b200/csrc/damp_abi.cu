@@ -21,6 +21,46 @@ struct damp_pool {
     PoolDesc d;
 };
 
+namespace damp {
+
+// Minimum-cost perfect matching of a head's 16 row groups, the cost of a pair
+// being the number of row positions where the two groups differ in format.
+// Exact, by dynamic programming over subsets of groups: the lowest group of a
+// subset is matched first, ties going to its lowest partner.  The pairs are
+// listed in ascending order of their lower group.
+void row_group_order(const uint32_t* mask, uint8_t order[16]) {
+    constexpr int G = 16;
+    uint8_t m[G];
+    for (int g = 0; g < G; ++g) m[g] = (uint8_t)(mask[g >> 2] >> (8 * (g & 3)));
+    std::vector<uint8_t> cost(1u << G, 0), pick(1u << G, 0);
+    for (uint32_t S = 1; S < (1u << G); ++S) {
+        if (__builtin_popcount(S) & 1) continue;
+        const int i = __builtin_ctz(S);
+        const uint32_t R = S & ~(1u << i);
+        int best = 1 << 30, bj = 0;
+        for (uint32_t T = R; T; T &= T - 1) {
+            const int j = __builtin_ctz(T);
+            const int c = __builtin_popcount((unsigned)(m[i] ^ m[j])) + cost[R & ~(1u << j)];
+            if (c < best) {
+                best = c;
+                bj = j;
+            }
+        }
+        cost[S] = (uint8_t)best;
+        pick[S] = (uint8_t)bj;
+    }
+    uint32_t S = (1u << G) - 1;
+    for (int k = 0; S; ++k) {
+        const int i = __builtin_ctz(S);
+        const int j = pick[S];
+        order[2 * k] = (uint8_t)i;
+        order[2 * k + 1] = (uint8_t)j;
+        S &= ~((1u << i) | (1u << j));
+    }
+}
+
+}  // namespace damp
+
 namespace {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -216,8 +256,11 @@ int create_common(int format, int n_slots, int H, int d_k, int hp_rows,
                         e = (i8_off + r8 * (uint32_t)d_k) | ((4u * r8) << 16);
                         ++r8;
                     }
-                    dir[(size_t)h * damp::kDirWords + i] = e;
+                    dir[(size_t)h * damp::kDirStride + i] = e;
                 }
+                damp::row_group_order(masks.data() + (size_t)h * damp::kMaskWords,
+                                      reinterpret_cast<uint8_t*>(dir + (size_t)h * damp::kDirStride +
+                                                                 damp::kDirWords));
             }
         }
         cudaError_t e = cudaMemcpy(dev_buf, hdr.data(), hdr.size(), cudaMemcpyHostToDevice);
@@ -289,6 +332,12 @@ int damp_pool_create_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is
     }
     return create_common(DAMP_FMT_MIXED, n_slots, H, d_k, hp < 0 ? -1 : hp, masks, dev_buf,
                          buf_bytes, out);
+}
+
+int damp_pool_row_groups(const damp_pool* pool, int h, uint8_t* order) {
+    if (!pool || !order || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
+    damp::row_group_order(pool->d.host_masks + (size_t)h * damp::kMaskWords, order);
+    return DAMP_OK;
 }
 
 int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,

@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
                 continue;
             }
             if constexpr (QUANT) {
-                load_tile_gdir<D, FP8>(blk, a.dir + (size_t)h * kDirWords, r0, cg, x);
+                load_tile_gdir<D, FP8>(blk, a.dir + (size_t)h * kDirStride, r0, cg, x);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {

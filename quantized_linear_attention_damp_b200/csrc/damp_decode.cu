@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
                 bulk_g2s(smem_u32(st + a.st_alpha + lane * D * 4), a.alpha + (size_t)u * D, D * 4,
                          fb);
             if constexpr (QUANT)
-                bulk_g2s(smem_u32(st + a.st_dir + lane * D * 4), a.dir + (size_t)h * kDirWords,
+                bulk_g2s(smem_u32(st + a.st_dir + lane * D * 4), a.dir + (size_t)h * kDirStride,
                          D * 4, fb);
         }
     };

@@ -5,15 +5,17 @@
 // kernel in damp_decode.cu ("STEPQuant ...", Appendix Table C2 steps 1, 2,
 // 3, 6 on the DAMP row format); only the work decomposition differs.
 //
-// CTA of 8 warps.  Half-warp hh of warp w owns key rows [8g, 8g + 8) of the
-// unit, g = 2w + hh; a lane owns 8 columns, so one row takes 16 lanes.  Each
-// thread keeps its 8 x 8 tile in registers from dequantize to requantize, and
-// the per-row work (directory lookup, scale, k/q values, row maximum,
-// division, stores) is spread over 8 columns.  The two halves of a warp work
-// on different rows, so a format branch runs both paths, each for its half,
-// when the rows differ in format.  u = k^T S' is summed in the recursive
-// pairwise order: 8 rows per thread as a subtree, then the top four levels
-// over the 16 row groups.
+// CTA of 8 warps.  Half-warp k = 2w + hh of warp w owns key rows [8g, 8g + 8)
+// of the unit, g = order[k] from the head's row-group order in the pool header;
+// a lane owns 8 columns, so one row takes 16 lanes.  Each thread keeps its
+// 8 x 8 tile in registers from dequantize to requantize, and the per-row work
+// (directory lookup, scale, k/q values, row maximum, division, stores) is
+// spread over 8 columns.  The two halves of a warp work on different rows, so
+// a format branch runs both paths, each for its half, where the rows differ in
+// format; the order pairs groups whose FP16 rows line up, so that this is
+// rare.  u = k^T S' is summed in the recursive pairwise order: 8 rows per
+// thread as a subtree, then the top four levels over the 16 row groups by
+// group index, whichever half-warp computed them.
 //
 // Two CTAs share an SM whenever three stages fit in half of its shared
 // memory (4 stages at 27 FP16 rows): their barriers are independent, so one CTA's arithmetic fills the
@@ -42,6 +44,7 @@ constexpr int kPT = 256;       // threads (8 warps)
 constexpr int kPD = 128;       // d_k = d_v
 constexpr int kPR = 8;         // rows per thread
 constexpr int kPG = 16;        // row groups (half-warps)
+constexpr uint32_t kDirBytes = kDirStride * 4;   // directory + row-group order
 
 // Per-unit metadata written by the refill warp into the stage (32 bytes).
 struct PMeta {
@@ -176,7 +179,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             *reinterpret_cast<PMeta*>(st + a.st_meta) = m;
             const uint32_t fb = full_bar(stage);
             if (m.active == 1) {
-                mbar_arrive_expect_tx(fb, m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u) + 4u * kPD);
+                mbar_arrive_expect_tx(fb, m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u) + kDirBytes);
                 bulk_g2s(smem_u32(st), a.blocks + m.boff, m.bytes, fb);
                 const size_t io = (size_t)m.unit * kPD * ELT;
                 bulk_g2s(smem_u32(st + a.st_q), static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
                 if constexpr (KDA)
                     bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + (size_t)m.unit * kPD, kPD * 4, fb);
-                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirWords, kPD * 4, fb);
+                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirStride, kDirBytes, fb);
             } else {
                 mbar_arrive(fb);
             }
@@ -204,18 +207,17 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     if (warp == kIssueWarp)
         for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
 
-    // ---- consumers: half-warp hh of warp w owns row group 2w + hh
+    // ---- consumers: half-warp k = 2w + hh of warp w owns row group order[k] of
+    // the unit's head
     const int hh = lane >> 4;
     const int cg = lane & 15;           // columns 8cg .. 8cg+7
-    const int rg = warp * 2 + hh;       // row group
-    const int r0 = rg * kPR;            // rows r0 .. r0+7
 
     uint8_t* scratch = smem + a.scratch_off;
-    float* red_u = reinterpret_cast<float*>(scratch);   // [16][128]
-    float* red_w = red_u + kPG * kPD;                   // [16][128]
+    float* red_u = reinterpret_cast<float*>(scratch);   // [16][128], by row group
+    float* red_w = red_u + kPG * kPD;                   // [16][128], by row group
     float* delta_s = red_w + kPG * kPD;                 // [128]
-    float* cpart_s = delta_s + kPD;                     // [16]
-    float* rowbuf = cpart_s + kPG + rg * 16;            // this half-warp's 16 floats
+    float* cpart_s = delta_s + kPD;                     // [16], by row group
+    float* rowbuf = cpart_s + kPG + (warp * 2 + hh) * 16;   // this half-warp's 16 floats
 
     int it = 0, stage = 0;
     uint32_t parity = 0;
@@ -225,6 +227,9 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
         const PMeta meta = *reinterpret_cast<const PMeta*>(st + a.st_meta);
         const bool any = ok && meta.active == 1;
+        // row group of this half-warp (the order is loaded with the directory)
+        const int rg = any ? (st[a.st_dir + kDirWords * 4 + warp * 2 + hh] & (kPG - 1)) : warp * 2 + hh;
+        const int r0 = rg * kPR;            // rows r0 .. r0+7
         uint8_t* blk = st;
         const uint8_t* sq = st + a.st_q;
         const uint8_t* sk = st + a.st_k;
@@ -471,7 +476,7 @@ uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
     off += kda ? kPD * 4 : 0;
     a.st_mask = off;
     a.st_dir = off;
-    off += kPD * 4;
+    off += kDirBytes;
     a.st_meta = off;
     off += sizeof(PMeta);
     a.stage_bytes = up(off, 128);

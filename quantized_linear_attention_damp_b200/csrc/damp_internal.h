@@ -9,7 +9,8 @@ namespace damp {
 // Header written at the start of the caller's pool buffer:
 //   [0, 16)                      device status word (uint32) + padding
 //   [16, 16 + 16*H)              per-head FP16-row masks, 4 x uint32 (key rows 0..127)
-//   [dir_off, dir_off + 512*H)   per-head row directory, 128 x uint32 (see below)
+//   [dir_off, dir_off + 528*H)   per-head row directory, 128 x uint32 (see below),
+//                                then the head's row-group order (16 bytes)
 //   [head_off, head_off + 16*H)  per-head block table, uint4 {block offset inside
 //                                the slot, block stride, FP16-row offset, INT8-row
 //                                offset} (heads may hold different FP16-row counts)
@@ -20,12 +21,22 @@ namespace damp {
 //   bits  0..15  byte offset of the row inside the block
 //   bits 16..30  byte offset of the row's FP32 scale (INT8 rows; 0 for FP16 rows)
 //   bit  31      1 = FP16 row, 0 = INT8 row
+//
+// Row-group order (read by the d = 128 decode kernel): byte k is the group g
+// of key rows [8g, 8g + 8) that half-warp k takes.  Half-warps 2w and 2w + 1
+// share warp w, and its format branches diverge on every row position where
+// their two groups differ in format; the order pairs the groups so that the
+// pairs differ in as few positions as possible (row_group_order).
 constexpr size_t kStatusBytes = 16;
 constexpr int kMaskWords = 4;
 constexpr int kMaxD = 128;
-constexpr int kDirWords = 128;
+constexpr int kDirWords = 128;               // directory entries per head
+constexpr int kDirStride = kDirWords + 4;    // words per head: entries + row-group order
 inline size_t dir_offset(int H) { return (kStatusBytes + (size_t)H * kMaskWords * 4 + 15) / 16 * 16; }
-inline size_t head_table_offset(int H) { return dir_offset(H) + (size_t)H * kDirWords * 4; }
+inline size_t head_table_offset(int H) { return dir_offset(H) + (size_t)H * kDirStride * 4; }
+
+// Row-group order of a head from its FP16-row mask (4 words, key rows 0..127).
+void row_group_order(const uint32_t* mask, uint8_t order[16]);
 
 struct PoolDesc {
     int format;      // DAMP_FMT_*

@@ -80,8 +80,8 @@ def test_layouts_of_other_formats():
 def test_pool_bytes():
     n = D.damp_pool_bytes(D.DAMP_FMT_MIXED, 64, 32, 128, 128, 27)
     # status word; per head a 16-byte FP16-row mask, a 512-byte row directory
-    # and a 16-byte block-table entry
-    hdr = 256 * ((16 + 32 * 16 + 32 * 512 + 32 * 16 + 255) // 256)
+    # followed by its 16-byte row-group order, and a 16-byte block-table entry
+    hdr = 256 * ((16 + 32 * 16 + 32 * (512 + 16) + 32 * 16 + 255) // 256)
     assert n == hdr + 64 * 32 * 20256
 
 
@@ -229,3 +229,66 @@ def test_validate_slots():
         with pytest.raises(D.DampError) as ei:
             D.damp_validate_slots(bad, 6)
         assert ei.value.status == D.DAMP_ERR_INVALID_ARGUMENT and f"entry {pos}" in str(ei.value)
+
+
+def _group_masks(is16_row):
+    return [int(sum(int(is16_row[8 * g + i]) << i for i in range(8))) for g in range(16)]
+
+
+def _pair_cost(m, order):
+    return sum(bin(m[order[2 * k]] ^ m[order[2 * k + 1]]).count("1") for k in range(8))
+
+
+def _min_pair_cost(m):
+    """Minimum over all perfect matchings of the 16 groups, by recursion over
+    the lowest unmatched group (memoised on the set of matched groups)."""
+    import functools
+
+    @functools.lru_cache(None)
+    def f(left):
+        if not left:
+            return 0
+        i, rest = left[0], left[1:]
+        return min(bin(m[i] ^ m[j]).count("1") + f(rest[:t] + rest[t + 1:])
+                   for t, j in enumerate(rest))
+    return f(tuple(range(16)))
+
+
+def test_row_group_order_is_a_minimum_cost_pairing():
+    """The d = 128 decode step's row-group order: a permutation of the 16
+    groups whose warp pairs differ in format at the fewest row positions."""
+    g = np.random.default_rng(7)
+    H, d = 6, 128
+    m = np.zeros((H, d), np.uint8)
+    for head, c in enumerate([0, 1, 27, 40, 64, 128]):
+        m[head, g.choice(d, c, replace=False)] = 1
+    h = D.damp_pool_create_map(3, H, d, d, m, None)
+    try:
+        for head in range(H):
+            order = D.damp_pool_row_groups(h, head)
+            assert sorted(order) == list(range(16))
+            gm = _group_masks(m[head])
+            assert _pair_cost(gm, order) == _min_pair_cost(gm)
+            lows = [min(order[2 * k], order[2 * k + 1]) for k in range(8)]
+            assert lows == sorted(lows) and all(order[2 * k] < order[2 * k + 1] for k in range(8))
+        # no FP16 row, or every row FP16: nothing to pair, groups in order
+        assert D.damp_pool_row_groups(h, 0) == list(range(16))
+        assert D.damp_pool_row_groups(h, 5) == list(range(16))
+        with pytest.raises(D.DampError):
+            D.damp_pool_row_groups(h, H)
+    finally:
+        D.damp_pool_destroy(h)
+
+
+def test_row_group_order_worked_example():
+    """Groups 0 and 2 hold FP16 rows at the same 8 positions, all others none:
+    0 pairs with 2 at no cost, then 1 with its lowest free partner 3, and the
+    rest in order."""
+    row = np.zeros(128, np.uint8)
+    row[0:8] = 1
+    row[16:24] = 1
+    h = D.damp_pool_create_map(1, 1, 128, 128, row[None, :], None)
+    try:
+        assert D.damp_pool_row_groups(h, 0) == [0, 2, 1, 3] + list(range(4, 16))
+    finally:
+        D.damp_pool_destroy(h)
