@@ -31,7 +31,15 @@ namespace damp {
 void row_group_order(const uint32_t* mask, uint8_t order[16]) {
     constexpr int G = 16;
     uint8_t m[G];
-    for (int g = 0; g < G; ++g) m[g] = (uint8_t)(mask[g >> 2] >> (8 * (g & 3)));
+    bool same = true;
+    for (int g = 0; g < G; ++g) {
+        m[g] = (uint8_t)(mask[g >> 2] >> (8 * (g & 3)));
+        same = same && m[g] == m[0];
+    }
+    if (same) {   // every pairing costs 0: the groups in order (what the search returns)
+        for (int g = 0; g < G; ++g) order[g] = (uint8_t)g;
+        return;
+    }
     std::vector<uint8_t> cost(1u << G, 0), pick(1u << G, 0);
     for (uint32_t S = 1; S < (1u << G); ++S) {
         if (__builtin_popcount(S) & 1) continue;
