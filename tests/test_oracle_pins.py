@@ -372,3 +372,78 @@ def test_update_is_one_rounding_of_the_exact_value():
             two_step = np.float32(np.float32(beta * delta[j]) + S[0, j])
             hits += int(two_step != ref)
     assert hits > 0   # the case does separate one rounding from two
+
+
+# ---------------------------------------------------------------- batch slot gather
+
+def _gather_case(seed, dk, dv, kda):
+    """A pool of 6 slots x 2 heads and a batch of 4 entries whose slot
+    indices are permuted, with one padding entry: entry b steps slot
+    slot_idx[b], which differs from b for every stepped entry."""
+    g = np.random.default_rng(seed)
+    n_slots, H = 6, 2
+    S = (g.standard_normal((n_slots, H, dk, dv))
+         * np.exp(g.standard_normal((n_slots, H, dk, 1)))).astype(np.float32)
+    slot_idx = np.int32([4, -1, 0, 5])
+    n = slot_idx.size
+    q = g.standard_normal((n, H, dk))
+    k = g.standard_normal((n, H, dk))
+    q = (q / np.linalg.norm(q, axis=-1, keepdims=True)).astype(np.float32)
+    k = (k / np.linalg.norm(k, axis=-1, keepdims=True)).astype(np.float32)
+    v = g.standard_normal((n, H, dv)).astype(np.float32)
+    alpha = g.uniform(0.5, 1.0, (n, H, dk) if kda else (n, H)).astype(np.float32)
+    beta = g.uniform(0.1, 1.0, (n, H)).astype(np.float32)
+    return S, slot_idx, q, k, v, alpha, beta
+
+
+@pytest.mark.parametrize("kda", [False, True])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (16, 32)])
+def test_batch_step_gathers_each_entry_slot(kda, dk, dv):
+    """Entry b reads and writes pool slot slot_idx[b] with entry b's inputs:
+    each stepped slot and each readout o[b] equal the FP64 brute force of the
+    matrix form applied to that slot's own pre-state and entry b's inputs;
+    the padding entry reads out zeros and slots nobody stepped keep their
+    bytes.  (Swapping the entry and slot indices anywhere in the batch step
+    fails here: every stepped slot differs from its entry.)"""
+    S, slot_idx, q, k, v, alpha, beta = _gather_case(91 + dk + dv + kda, dk, dv, kda)
+    n_slots, H = S.shape[:2]
+    gate = O.GATE_VECTOR if kda else O.GATE_SCALAR
+    pool = O.pack(O.FMT_FP32, np.zeros((H, dk)), S)
+    o = O.decode_step(pool, gate, np.zeros((H, dk), np.uint8), slot_idx, q, k, v, alpha, beta)
+    stepped = set()
+    for b, slot in enumerate(slot_idx):
+        if slot < 0:
+            assert not o[b].any()
+            continue
+        stepped.add(int(slot))
+        for h in range(H):
+            Sn, on = BF.step(S[slot, h], q[b, h], k[b, h], v[b, h], alpha[b, h], beta[b, h])
+            assert np.max(np.abs(pool.f32[slot, h] - Sn)) <= 1e-5 * np.max(np.abs(Sn)), (b, h)
+            assert np.max(np.abs(o[b, h] - on)) <= 1e-5 * max(1.0, np.max(np.abs(on))), (b, h)
+    for slot in range(n_slots):
+        if slot not in stepped:
+            assert np.array_equal(pool.f32[slot].view(np.uint32), S[slot].view(np.uint32))
+
+
+def test_batch_step_gather_quantized_matches_unit_steps():
+    """Mixed format: the batch step equals unit steps taken on the slot that
+    each entry names, bit for bit (the unit step is pinned on its own above)."""
+    S, slot_idx, q, k, v, alpha, beta = _gather_case(97, 32, 32, False)
+    n_slots, H, dk, dv = S.shape
+    g = np.random.default_rng(98)
+    flags = np.zeros((H, dk), np.uint8)
+    for h in range(H):
+        flags[h, g.permutation(dk)[:7]] = 1
+    pool = O.pack(O.FMT_QUANT, flags[None], S)
+    ref = pool.copy()
+    o = O.decode_step(pool, O.GATE_SCALAR, flags, slot_idx, q, k, v, alpha, beta)
+    for b, slot in enumerate(slot_idx):
+        if slot < 0:
+            continue
+        for h in range(H):
+            ou = O.step_unit(ref[slot, h], O.GATE_SCALAR, flags[h], q[b, h], k[b, h], v[b, h],
+                             alpha[b, h], beta[b, h])
+            assert np.array_equal(o[b, h], ou)
+    for f in ("scale", "half", "code"):
+        assert np.array_equal(getattr(pool, f), getattr(ref, f))
+    assert not np.array_equal(pool.code[4], O.pack(O.FMT_QUANT, flags[None], S).code[4])
