@@ -303,6 +303,33 @@ int damp_calib_select(int H, int d_k, int hp_rows, const double* acc, double* sc
 int damp_calib_select_budget(int H, int d_k, int budget, const double* acc, double* score,
                              uint8_t* is_fp16, int32_t* hp_per_head, void* stream);
 
+/*
+ * damp_calib_select_budget without the caller's score buffer, for callers that
+ * cannot allocate device memory when they select: a serving process whose
+ * memory plan hands all free HBM to the state pools up front, or a C host
+ * with no allocator of its own that only holds buffers it was given.  (The
+ * pages have no counterpart: this is an interface convenience, not part of
+ * the method.)
+ *
+ * The scores go to a scratch array inside the library instead: one static
+ * device array of DAMP_SELECT_BUDGET_STATIC_MAX doubles (128 KiB), which every
+ * GPU that loads the library holds until the process exits.  The call
+ * allocates and frees nothing.  Results (is_fp16, hp_per_head) are the same
+ * as damp_calib_select_budget's; no scores are returned.
+ *   - H * d_k > DAMP_SELECT_BUDGET_STATIC_MAX: DAMP_ERR_UNSUPPORTED, nothing
+ *     enqueued.  Other arguments as for damp_calib_select_budget.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array, and it keeps the last
+ *     call's scores (each call writes every entry it reads first).  Calls
+ *     whose work overlaps on the GPU (different streams, no ordering between
+ *     them) race on it: order them on one stream or with events.
+ */
+#define DAMP_SELECT_BUDGET_STATIC_MAX 16384
+int damp_calib_select_budget_static(int H, int d_k, int budget, const double* acc,
+                                    uint8_t* is_fp16, int32_t* hp_per_head, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

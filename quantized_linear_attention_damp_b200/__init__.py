@@ -80,6 +80,7 @@ def _load():
         "damp_calib_accumulate": (I, [P, I, P, I, P, P, P]),
         "damp_calib_select": (I, [I, I, I, P, P, P, P]),
         "damp_calib_select_budget": (I, [I, I, I, P, P, P, P, P]),
+        "damp_calib_select_budget_static": (I, [I, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -354,6 +355,29 @@ def damp_calib_select_budget(H: int, d_k: int, budget: int, acc: torch.Tensor, s
                                          _ptr(hp), _stream(stream, acc.device)),
            "damp_calib_select_budget")
     return is16, hp, score
+
+
+DAMP_SELECT_BUDGET_STATIC_MAX = 16384
+
+
+def damp_calib_select_budget_static(H: int, d_k: int, budget: int, acc: torch.Tensor,
+                                    is_fp16: torch.Tensor, hp_per_head: torch.Tensor,
+                                    stream=None) -> None:
+    """Budget selection that allocates nothing: for callers that cannot
+    allocate device memory at selection time (every free byte already handed
+    to the state pools, or a host with no allocator that only holds buffers
+    it was given).  The caller passes the outputs, is_fp16 uint8 [H][d_k] and
+    hp_per_head int32 [H]; the scores go to the library's static device array
+    (H * d_k <= DAMP_SELECT_BUDGET_STATIC_MAX).  Calls that overlap on the GPU
+    share that array and race: keep them on one stream."""
+    _cuda(acc, torch.float64, "acc")
+    _cuda(is_fp16, torch.uint8, "is_fp16")
+    _cuda(hp_per_head, torch.int32, "hp_per_head")
+    if is_fp16.numel() != H * d_k or hp_per_head.numel() != H:
+        raise ValueError("is_fp16 must hold H*d_k bytes and hp_per_head H entries")
+    _check(_lib.damp_calib_select_budget_static(H, d_k, budget, _ptr(acc), _ptr(is_fp16),
+                                                _ptr(hp_per_head), _stream(stream, acc.device)),
+           "damp_calib_select_budget_static")
 
 
 # ---------------------------------------------------------------- convenience

@@ -13,6 +13,8 @@
 // loaded before any is reduced to keep several row reads in flight per warp.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "damp.h"
 #include "damp_device.cuh"
 #include "damp_internal.h"
@@ -219,3 +221,60 @@ cudaError_t launch_calib_select_budget(const double* acc, int H, int d, int budg
 }
 
 }  // namespace damp
+
+// ---------------------------------------------------------------------------
+// Budget selection with library-owned scratch: the scores live in a static
+// device array instead of a caller buffer, so the call allocates nothing.
+// ---------------------------------------------------------------------------
+namespace damp {
+namespace {
+
+constexpr int kStaticScores = DAMP_SELECT_BUDGET_STATIC_MAX;   // 128 KiB of doubles
+
+// Every device that loads the library holds one copy until the process exits.
+static __device__ __align__(256) double g_budget_scores[kStaticScores];
+
+// Device address of g_budget_scores on each device, looked up once per device
+// with that device current (in host code the symbol itself is only a host-side
+// stand-in and must never reach a kernel).
+constexpr int kMaxDevices = 64;
+std::mutex g_scores_mu;
+double* g_scores_addr[kMaxDevices] = {};
+
+cudaError_t static_scores(double** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scores_mu);
+    if (!g_scores_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_budget_scores);
+        if (e != cudaSuccess) return e;
+        g_scores_addr[dev] = static_cast<double*>(p);
+    }
+    *out = g_scores_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace damp
+
+extern "C" int damp_calib_select_budget_static(int H, int d_k, int budget, const double* acc,
+                                               uint8_t* is_fp16, int32_t* hp_per_head,
+                                               void* stream) {
+    if (H <= 0 || d_k <= 0) return DAMP_ERR_INVALID_ARGUMENT;
+    if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return DAMP_ERR_UNSUPPORTED;
+    if ((size_t)H * d_k > (size_t)damp::kStaticScores) return DAMP_ERR_UNSUPPORTED;
+    if (budget < 0 || budget > H * d_k || !acc || !is_fp16 || !hp_per_head)
+        return DAMP_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(acc) & 7u) || (reinterpret_cast<uintptr_t>(hp_per_head) & 3u))
+        return DAMP_ERR_MISALIGNED;
+    double* scores = nullptr;
+    if (damp::static_scores(&scores) != cudaSuccess) return DAMP_ERR_CUDA;
+    const cudaError_t e = damp::launch_calib_select_budget(acc, H, d_k, budget, scores, is_fp16,
+                                                           hp_per_head,
+                                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DAMP_OK : DAMP_ERR_CUDA;
+}
+
