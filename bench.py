@@ -4,12 +4,14 @@
 
 A step is one decode step (dequantize, gated delta rule, readout,
 requantize in place) over every (slot, head) of the workload, i.e. one
-launch of the decode kernel.  The default workload is the 64-slot x 32-head
-GDN batch at d = 128 with 27 FP16 rows per head (9.885 bits/value).  Its state
-(41.5 MB) fits in L2, so consecutive steps rotate over several pools and input
-sets totalling at least 4x L2 (every step reads cold state and pays for
-earlier write-backs); each step is timed with CUDA events on the launching
-stream and the durations are summed.
+launch of the decode kernel.  The default workload is the 512-slot x 48-head
+GDN batch at d = 128 with 27 FP16 rows per head (9.885 bits/value, bf16 q/k/v):
+the batch >= 256, d = 128 point the throughput target is stated for.  Lines
+for the 256-slot x 32-head GDN batch and the 128-slot x 32-head KDA batch are
+printed beside it (`sub_lines`, same keys).  Consecutive steps rotate over
+enough pools and input sets to touch at least 4x L2 (every step reads cold
+state and pays for earlier write-backs); each step is timed with CUDA events
+on the launching stream and the durations are summed.
 
 Printed: one JSON line (rank 0).  `value` is head-steps/s over all ranks;
 `roofline` is the decode kernel's algorithmic bytes per launch over its mean
@@ -40,7 +42,7 @@ import workloads as W  # noqa: E402
 METRIC = "head-steps/s and achieved HBM GB/s (% of B200 roofline) per decode step"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["damp_decode_unit.cu", "damp_device.cuh", "damp_internal.h"]   # the profiled kernel
-PROFILE = os.path.join(ROOT, "profiles", "decode_unit_hiconc_gdn_mixed.txt")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 
 # ---------------------------------------------------------------- accounting
@@ -78,12 +80,13 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units: int):
-    """DRAM bytes per launch from the committed ncu summary, scaled to this
+def profiled_traffic(w: W.Workload, fmt: str, units: int):
+    """DRAM bytes per launch from the committed ncu summary of this workload
+    and format (profiles/decode_unit_<workload>_<fmt>.txt), scaled to this
     launch's units; None if absent or taken on different kernel sources."""
     try:
         kv = {}
-        for line in open(PROFILE):
+        for line in open(os.path.join(PROFILE_DIR, f"decode_unit_{w.name}_{fmt}.txt")):
             if ":" in line:
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
@@ -249,6 +252,9 @@ class Bench:
               for _ in range(steps)]
         ctx = sampler if sampler is not None else _Null()
         with ctx:
+            # keep the device busy while the host enqueues the timed steps, so
+            # that the events time the kernels and not the host's launch rate
+            torch.cuda._sleep(min(steps, 4000) * 200_000)
             for i in range(steps):
                 ev[i][0].record()
                 self.step(warmup + i)
@@ -327,68 +333,101 @@ def cpu_baseline_threads(w: W.Workload, fmt: str, seconds: float, threads: int):
     return n / el, n, el
 
 
-def run_native(args, rank, world, local_rank):
+def config_of(w: W.Workload, fmt: str, world: int, l2: str, timing: str) -> dict:
+    """The workload description shared by both arms (same keys)."""
+    return {"workload": describe(w, fmt), "units_per_step_per_gpu": w.n * w.H,
+            "algorithmic_bytes_per_unit": unit_bytes(w, fmt), "l2": l2, "timing": timing,
+            "parallelism": f"dp{world} (slots sharded, no collective)"}
+
+
+def measure(w: W.Workload, fmt: str, dev, steps: int, warmup: int, world: int = 1,
+            local_rank: int = 0, cpu_seconds: float = 0.0, e2e: bool = True) -> dict:
+    """One workload's line: device-timed steps (max over ranks), roofline of
+    the decode kernel, clocks during the timed region, the same steps end to
+    end through the public API, and the oracle on the host cores."""
     import torch
     import torch.distributed as dist
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = rank_workload(args.workload, rank)
-    fmt = args.fmt
     b = Bench(w, fmt, device=dev)
     units = w.n * w.H
     ub = unit_bytes(w, fmt)
-
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(local_rank)
-    secs = max_over_ranks(b.timed(args.steps, args.warmup, sampler), world, dev)
+    secs = max_over_ranks(b.timed(steps, warmup, sampler), world, dev)
     if world > 1:
         dist.barrier()
-    e2e_secs, h2d, d2h = (b.timed_e2e(args.steps) if not args.no_e2e else (float("nan"), 0, 0))
+    e2e_secs, h2d, d2h = b.timed_e2e(steps) if e2e else (float("nan"), 0, 0)
     e2e_secs = max_over_ranks(e2e_secs, world, dev)
     b.close()
-
-    if rank != 0:
-        return
-    per_launch = secs / args.steps
-    value = units * world * args.steps / secs
+    per_launch = secs / steps
     gbs = ub * units / per_launch / 1e9
     peak, src = measured_peak()
     line = {
-        "metric": METRIC, "value": value, "unit": "head-steps/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_launch * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "config": {"workload": describe(w, fmt), "units_per_step_per_gpu": units,
-                   "algorithmic_bytes_per_unit": ub,
-                   "l2": f"steps rotate over {b.n_pools} pools ({b.touched_bytes / 1e6:.0f} MB) "
-                         "and their inputs, >= 4x L2: inputs larger than L2",
-                   "timing": "CUDA events around each step on the launch stream, summed",
-                   "parallelism": f"dp{world} (slots sharded, no collective)"},
+        "value": units * world * steps / secs, "unit": "head-steps/s",
+        "ms_per_step": per_launch * 1e3,
+        "config": config_of(w, fmt, world,
+                            l2=f"steps rotate over {b.n_pools} pools "
+                               f"({b.touched_bytes / 1e6:.0f} MB) and their inputs, >= 4x L2: "
+                               "inputs larger than L2",
+                            timing="CUDA events around each step on the launch stream, summed"),
         "hbm_gbs": gbs,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                      "frac": gbs / peak, "peak_source": src,
                      "frac_of_8tbs_nominal": gbs / 8000.0,
-                     "traffic": profiled_traffic(units)},
+                     "traffic": profiled_traffic(w, fmt, units)},
         "step_us": {"median": b.step_ms[len(b.step_ms) // 2] * 1e3, "min": b.step_ms[0] * 1e3},
-        "gpu_launches": args.steps,
+        "gpu_launches": steps,
         "clocks": sampler.summary(),
-        "e2e": ({"value": units * world * args.steps / e2e_secs, "unit": "head-steps/s",
-                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-                if not args.no_e2e else None),
+        "e2e": ({"value": units * world * steps / e2e_secs, "unit": "head-steps/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h} if e2e else None),
     }
-    if world == 1 and args.cpu_seconds > 0:
-        v, n, el = cpu_baseline(w, fmt, args.cpu_seconds)
+    if world == 1 and cpu_seconds > 0:
+        v, n, el = cpu_baseline(w, fmt, cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "head-steps/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{n} (slot, head) units of {w.name} ({fmt}), "
                                           f"one step each, single thread, {el:.1f} s"}
+    return line
+
+
+# sub-lines printed beside the headline: the other d = 128 target points
+SUB_LINES = [("gdn_256x32", "mixed"), ("kda", "mixed")]
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = rank_workload(args.workload, rank)
+    fmt = args.fmt
+    head = measure(w, fmt, dev, args.steps, args.warmup, world, local_rank,
+                   args.cpu_seconds if world == 1 else 0.0, e2e=not args.no_e2e)
+    subs = []
+    if not args.no_sub_lines:
+        for name, sfmt in SUB_LINES:
+            if name == args.workload and sfmt == fmt:
+                continue
+            sl = measure(rank_workload(name, rank), sfmt, dev, args.steps, args.warmup, world,
+                         local_rank, min(args.cpu_seconds, 3.0) if world == 1 else 0.0,
+                         e2e=not args.no_e2e)
+            sl["metric"] = METRIC
+            subs.append(sl)
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": head["value"], "unit": "head-steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic"}
+    line.update({k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step")})
+    if world == 1 and args.cpu_seconds > 0:
         t = os.cpu_count() or 1
         v, n, el = cpu_baseline_threads(w, fmt, args.cpu_seconds, t)
         line["cpu_baseline_all_cores"] = {
             "value": v, "unit": "head-steps/s", "cores": t, "kind": "oracle",
             "sample": f"{n} (slot, head) units of {w.name} ({fmt}), one step each, "
                       f"{t} threads over units (the oracle's C calls release the GIL), {el:.1f} s"}
+    if subs:
+        line["sub_lines"] = subs
     if world == 1 and not args.no_variants:
         line["variants"] = variants(args, dev)
     if world == 1 and not args.no_variants:
@@ -402,9 +441,8 @@ def variants(args, dev):
     """Context: the same kernel on the other workloads and state formats."""
     res = []
     steps = max(20, min(args.steps, 200))
-    for name, fmt in [("gdn_256x32", "mixed"), ("kda", "mixed"), ("hiconc_gdn", "mixed"),
-                      ("hiconc_gdn", "int8"), ("hiconc_gdn", "fp8"), ("hiconc_gdn", "fp32"),
-                      ("gdn_batch", "int8"), ("gdn_batch", "fp32")]:
+    for name, fmt in [("hiconc_gdn", "int8"), ("hiconc_gdn", "fp8"), ("hiconc_gdn", "fp32"),
+                      ("gdn_batch", "mixed"), ("gdn_batch", "int8"), ("gdn_batch", "fp32")]:
         w = W.WORKLOADS[name]
         b = Bench(w, fmt, device=dev)
         secs = b.timed(steps, 3)
@@ -667,8 +705,11 @@ def run_reference(args, rank, world):
         "ms_per_step": total_t / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": describe(w, fmt),
-                   "sample": f"{per_step} (slot, head) units per step of the {w.n * w.H}"},
+        "config": config_of(w, fmt, world,
+                            l2="host CPU run of the oracle: no GPU cache involved",
+                            timing="host wall clock (time.perf_counter) around the oracle's "
+                                   f"unit steps; each step a sample of {per_step} of the "
+                                   f"{w.n * w.H} (slot, head) units"),
         "cpu_baseline": {"value": value, "unit": "head-steps/s", "cores": 1, "kind": "oracle",
                          "sample": f"{per_step} units per step x {args.steps} steps, "
                                    "single thread"},
@@ -684,13 +725,15 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="gdn_batch", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default="hiconc_gdn", choices=list(W.WORKLOADS))
     ap.add_argument("--fmt", default="mixed", choices=["mixed", "int8", "fp8", "fp32"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-serving", action="store_true",
                     help="skip the 36-layer serving-pool context run (about 97 GB)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sub-lines", action="store_true",
+                    help="skip the 256x32 GDN and 128x32 KDA lines printed beside the headline")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

@@ -25,7 +25,12 @@
  *   u_j     = sum_i fl(k_i * S'_ij), recursive pairwise order over rows
  *   delta_j = fl(v_j - u_j);  b_i = fl(beta * k_i)
  *   X_ij    = fma(b_i, delta_j, S'_ij)           (all of the above in FP32)
- *   out_j   = sum_i q_i X_ij                     (FP32, from X, any order)
+ *   out_j   = X^T q read out before requantization, computed through the
+ *             identity X^T q = S'^T q + (q^T b) delta:  w = S'^T q and
+ *             c = q^T b (FP32, any order), out_j = fma(c, delta_j, w_j).  It
+ *             differs from sum_i q_i X_ij only by FP32 rounding (checked
+ *             against the FP64 readout of X within 1e-4 relative / 1e-5
+ *             absolute).
  *   FP16 rows: X rounded to binary16, nearest-even.
  *   INT8 rows: a = max_j |X_ij|; scale = fl(a/127); inv = fl(127/a);
  *              code = nearest integer to the exact X*inv, ties to even.
@@ -50,8 +55,9 @@
  *     see (a slot index out of range, an internal wait that hit its bound)
  *     set bits in the pool's status word (damp_pool_get_error); kernels never
  *     trap.
- *   - Supported shapes: d_k == d_v == d, d in {16, 32, 64, 128}; 1 <= H;
- *     1 <= n_slots; 0 <= hp_rows <= d_k.
+ *   - Supported shapes: d_k and d_v multiples of 16 in [16, 256] (d_k may
+ *     differ from d_v); 1 <= H; 1 <= n_slots; 0 <= hp_rows <= d_k.  The
+ *     square shapes d_k = d_v in {16, 32, 64, 128} run the fastest kernels.
  *   - Device pointers passed for bulk copies (pool buffer, q, k, v, KDA
  *     alpha, out, FP32 states) must be 16-byte aligned.
  */
@@ -77,6 +83,8 @@ extern "C" {
 /* ---- device status word bits (damp_pool_get_error) ----------------------- */
 #define DAMP_EFLAG_SLOT_RANGE 1u /* a slot_idx entry >= n_slots (entry skipped) */
 #define DAMP_EFLAG_TIMEOUT 2u    /* an internal pipeline wait hit its bound     */
+#define DAMP_EFLAG_NONFINITE 4u  /* a unit's inputs held a NaN or an infinity
+                                    (damp_decode_step_validated; unit skipped) */
 
 /* ---- enums ----------------------------------------------------------------- */
 #define DAMP_FMT_FP32 0     /* plain FP32 state (the pages' unquantized baseline)   */
@@ -115,8 +123,8 @@ int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
 
 /*
  * Bytes the caller must allocate for a pool of n_slots x H blocks: a header
- * (device status word, per-head FP16-row masks, row directory with the
- * row-group order, and block table, 256 B aligned) followed by the slots.  With one FP16-row count for
+ * (device status word, per-head FP16-row masks, row directory and block
+ * table, 256 B aligned) followed by the slots.  With one FP16-row count for
  * every head, block (slot, h) is at header + (slot*H + h)*stride.
  */
 int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
@@ -158,18 +166,6 @@ int damp_pool_create_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is
  * Any output pointer may be NULL. */
 int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,
                           size_t* block_stride, size_t* offset_in_slot);
-
-/*
- * Head h's row-group order, as the d = 128 decode step uses it (a work
- * decomposition only: results do not depend on it).  The kernel gives each
- * half-warp one group of 8 consecutive key rows, two groups per warp; a warp
- * whose two groups differ in format at a row position runs both format paths
- * there.  order[16] (host) receives the groups g (rows 8g .. 8g+7) in
- * half-warp order, paired so that the number of such positions over the
- * head is the minimum over all pairings (exact; ties to the lower group).
- * The pool header stores the same order after the head's row directory.
- */
-int damp_pool_row_groups(const damp_pool* pool, int h, uint8_t* order);
 
 /* Release the descriptor (never the caller's device buffer).  NULL is a no-op. */
 int damp_pool_destroy(damp_pool* pool);
@@ -216,6 +212,36 @@ int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int 
                      const float* alpha, const float* beta, float* out, void* stream);
 
 /*
+ * damp_decode_step with the inputs of every unit checked on the device: a
+ * unit whose q, k, v, alpha or beta holds a NaN or an infinity is skipped
+ * (its out row is zeroed, its block is neither updated nor stored) and
+ * DAMP_EFLAG_NONFINITE is set in the pool's status word.  Nothing traps.
+ * The pages leave non-finite inputs undefined (the oracle does not model
+ * them); this variant is for callers that want them caught instead of
+ * propagated into the stored state.  Same arguments and results otherwise.
+ */
+int damp_decode_step_validated(const damp_pool* pool, int n, const int32_t* slot_idx,
+                               int in_dtype, const void* q, const void* k, const void* v,
+                               int gate, const float* alpha, const float* beta, float* out,
+                               void* stream);
+
+/*
+ * Test hooks of the failure path (for tests of the library; not for serving).
+ *   wait_limit_ns : bound of every internal pipeline wait of the decode step;
+ *                   0 restores the default (2 s).  A wait that runs out sets
+ *                   DAMP_EFLAG_TIMEOUT in the pool's status word; the kernel
+ *                   then waits (bounded) for its copies in flight and returns,
+ *                   so the CUDA context stays usable.
+ *   hooks         : 0, or DAMP_HOOK_HOLD_FIRST_ITEM: every CTA of the decode
+ *                   step leaves the loads of its first work item unissued, so
+ *                   the wait for them runs out; no unit of the call is
+ *                   updated or stored and the out rows are left as they were.
+ * Process-wide, for the launches enqueued after the call.
+ */
+#define DAMP_HOOK_HOLD_FIRST_ITEM 1u
+int damp_set_test_hooks(uint64_t wait_limit_ns, uint32_t hooks);
+
+/*
  * Host-side check of a batch's slot indices (host int32 array [n]), for
  * callers that want it before a step: every non-negative entry must be below
  * n_slots and appear once.  Duplicates would give one block two writers in
@@ -246,6 +272,20 @@ int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float
 int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
                             const uint16_t* half, const int8_t* code, const float* f32,
                             void* block);
+
+/*
+ * Block (slot, h) of a pool in its logical per-row form, read from the device
+ * into host memory (for tests and inspection, not the serving path: a
+ * blocking device-to-host copy on the legacy default stream).  host_out
+ * receives, rows in key-channel order:
+ *   FP32 pools:      f32[d_k][d_v]                                    (4*d_k*d_v bytes)
+ *   quantized pools: scale[d_k] (float), then half[d_k][d_v] (uint16),
+ *                    then code[d_k][d_v] (int8), as damp_block_to_logical
+ *                    fills them                             (4*d_k + 3*d_k*d_v bytes)
+ * The caller owns host_out.  DAMP_ERR_INVALID_ARGUMENT for a host-only
+ * descriptor or an index out of range; DAMP_ERR_CUDA if the copy fails.
+ */
+int damp_pool_read_raw(const damp_pool* pool, int slot, int h, void* host_out);
 
 /* ---- offline calibration of the FP16 key rows ------------------------------
  *

@@ -30,6 +30,8 @@ DAMP_ERR_TIMEOUT = -6
 
 DAMP_EFLAG_SLOT_RANGE = 1
 DAMP_EFLAG_TIMEOUT = 2
+DAMP_EFLAG_NONFINITE = 4
+DAMP_HOOK_HOLD_FIRST_ITEM = 1
 
 DAMP_FMT_FP32 = 0
 DAMP_FMT_INT8_ROW = 1
@@ -67,6 +69,8 @@ def _load():
         "damp_pool_pack": (I, [P, I, P, P, P]),
         "damp_pool_unpack": (I, [P, I, P, P, P]),
         "damp_decode_step": (I, [P, I, P, I, P, P, P, I, P, P, P, P]),
+        "damp_decode_step_validated": (I, [P, I, P, I, P, P, P, I, P, P, P, P]),
+        "damp_set_test_hooks": (I, [ctypes.c_uint64, ctypes.c_uint32]),
         "damp_pool_get_error": (I, [P, ctypes.POINTER(ctypes.c_uint32), I, P]),
         "damp_block_to_logical": (I, [P, I, P, P, P, P, P]),
         "damp_block_from_logical": (I, [P, I, P, P, P, P, P]),
@@ -74,7 +78,7 @@ def _load():
         "damp_pool_create_map": (I, [I, I, I, I, P, P, S, ctypes.POINTER(P)]),
         "damp_pool_head_layout": (I, [P, I, ctypes.POINTER(S), ctypes.POINTER(S),
                                       ctypes.POINTER(S)]),
-        "damp_pool_row_groups": (I, [P, I, P]),
+        "damp_pool_read_raw": (I, [P, I, I, P]),
         "damp_validate_slots": (I, [P, I, I, ctypes.POINTER(I)]),
         "damp_calib_bytes": (S, [I, I]),
         "damp_calib_accumulate": (I, [P, I, P, I, P, P, P]),
@@ -95,6 +99,35 @@ _lib = _load()
 def _check(status: int, where: str):
     if status != DAMP_OK:
         raise DampError(status, where)
+
+
+# (format, n_slots, H, d_k, d_v) of every pool descriptor made through this
+# module: the C ABI cannot see tensor sizes, so the binding checks them
+# against the pool before anything is enqueued.
+_POOLS: dict[int, tuple[int, int, int, int, int]] = {}
+
+
+def _pool_shape(pool: int):
+    try:
+        return _POOLS[int(pool)]
+    except (KeyError, TypeError):
+        raise ValueError("unknown pool handle: create pools through this module") from None
+
+
+def _shape(t, name: str, shape: tuple):
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _same_device(stream, *tensors):
+    dev = tensors[0].device
+    for t in tensors[1:]:
+        if t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
+    if isinstance(stream, torch.cuda.Stream) and stream.device != dev:
+        raise ValueError(f"stream on {stream.device}, tensors on {dev}")
 
 
 def _ptr(t) -> int | None:
@@ -163,6 +196,7 @@ def damp_pool_create(format: int, n_slots: int, H: int, d_k: int, d_v: int, hp_r
     h = ctypes.c_void_p()
     _check(_lib.damp_pool_create(format, n_slots, H, d_k, d_v, hp_rows, _ptr(idx), buf_ptr,
                                  nbytes, ctypes.byref(h)), "damp_pool_create")
+    _POOLS[h.value] = (int(format), n_slots, H, d_k, d_v)
     return h.value
 
 
@@ -188,6 +222,7 @@ def damp_pool_create_map(n_slots: int, H: int, d_k: int, d_v: int, is_fp16, buf)
         ptr, nbytes = _ptr(buf), buf.numel()
     _check(_lib.damp_pool_create_map(n_slots, H, d_k, d_v, _ptr(m), ptr, nbytes,
                                      ctypes.byref(h)), "damp_pool_create_map")
+    _POOLS[h.value] = (DAMP_FMT_MIXED, n_slots, H, d_k, d_v)
     return h.value
 
 
@@ -199,16 +234,9 @@ def damp_pool_head_layout(pool: int, h: int) -> tuple[int, int, int]:
     return b.value, s.value, o.value
 
 
-def damp_pool_row_groups(pool: int, h: int) -> list[int]:
-    """Head h's row-group order: the group (key rows 8g .. 8g+7) of each
-    half-warp of the d = 128 decode step, two per warp."""
-    order = (ctypes.c_uint8 * 16)()
-    _check(_lib.damp_pool_row_groups(pool, h, order), "damp_pool_row_groups")
-    return list(order)
-
-
 def damp_pool_destroy(pool: int) -> None:
     _check(_lib.damp_pool_destroy(pool), "damp_pool_destroy")
+    _POOLS.pop(pool, None)
 
 
 def damp_pool_block_offset(pool: int, slot: int, h: int) -> int:
@@ -217,20 +245,39 @@ def damp_pool_block_offset(pool: int, slot: int, h: int) -> int:
     return o.value
 
 
-def damp_block_to_logical(pool: int, h: int, block, fmt: int, d: int) -> dict:
+def damp_block_to_logical(pool: int, h: int, block, fmt: int, d_k: int,
+                          d_v: int | None = None) -> dict:
     """Logical per-row form of one raw block (host bytes)."""
+    d_v = d_k if d_v is None else d_v
     block = np.ascontiguousarray(np.frombuffer(bytes(block), np.uint8))
     if fmt == DAMP_FMT_FP32:
-        f32 = np.empty((d, d), np.float32)
+        f32 = np.empty((d_k, d_v), np.float32)
         _check(_lib.damp_block_to_logical(pool, h, _ptr(block), None, None, None, _ptr(f32)),
                "damp_block_to_logical")
         return {"f32": f32}
-    scale = np.empty(d, np.float32)
-    half = np.empty((d, d), np.uint16)
-    code = np.empty((d, d), np.int8)
+    scale = np.empty(d_k, np.float32)
+    half = np.empty((d_k, d_v), np.uint16)
+    code = np.empty((d_k, d_v), np.int8)
     _check(_lib.damp_block_to_logical(pool, h, _ptr(block), _ptr(scale), _ptr(half), _ptr(code),
                                       None), "damp_block_to_logical")
     return {"scale": scale, "half": half, "code": code}
+
+
+def damp_pool_read_raw(pool: int, slot: int, h: int) -> dict:
+    """Block (slot, h) in its logical form, read from the device (host arrays:
+    f32 [d_k][d_v], or scale [d_k], half [d_k][d_v], code [d_k][d_v])."""
+    fmt, _, _, d_k, d_v = _pool_shape(pool)
+    if fmt == DAMP_FMT_FP32:
+        out = np.empty(4 * d_k * d_v, np.uint8)
+    else:
+        out = np.empty(4 * d_k + 3 * d_k * d_v, np.uint8)
+    _check(_lib.damp_pool_read_raw(pool, slot, h, _ptr(out)), "damp_pool_read_raw")
+    if fmt == DAMP_FMT_FP32:
+        return {"f32": out.view(np.float32).reshape(d_k, d_v)}
+    ne = d_k * d_v
+    return {"scale": out[:4 * d_k].view(np.float32).copy(),
+            "half": out[4 * d_k:4 * d_k + 2 * ne].view(np.uint16).reshape(d_k, d_v).copy(),
+            "code": out[4 * d_k + 2 * ne:].view(np.int8).reshape(d_k, d_v).copy()}
 
 
 def damp_block_from_logical(pool: int, h: int, stride: int, scale=None, half=None, code=None,
@@ -246,26 +293,49 @@ def damp_block_from_logical(pool: int, h: int, stride: int, scale=None, half=Non
 
 # ---------------------------------------------------------------- device calls
 
-def damp_pool_pack(pool: int, slot_idx: torch.Tensor, state: torch.Tensor, stream=None) -> None:
+def _codec_args(pool, slot_idx, state, stream, where):
+    _, _, H, d_k, d_v = _pool_shape(pool)
+    if not isinstance(slot_idx, torch.Tensor) or slot_idx.dim() != 1:
+        raise ValueError(f"{where}: slot_idx must be a 1-D tensor")
+    _shape(state, "state", (slot_idx.numel(), H, d_k, d_v))
     _cuda(slot_idx, torch.int32, "slot_idx")
     _cuda(state, torch.float32, "state")
+    _same_device(stream, slot_idx, state)
+
+
+def damp_pool_pack(pool: int, slot_idx: torch.Tensor, state: torch.Tensor, stream=None) -> None:
+    """Compress FP32 states [n][H][d_k][d_v] into the slots slot_idx [n]."""
+    _codec_args(pool, slot_idx, state, stream, "damp_pool_pack")
     _check(_lib.damp_pool_pack(pool, slot_idx.numel(), _ptr(slot_idx), _ptr(state),
                                _stream(stream, state.device)), "damp_pool_pack")
 
 
 def damp_pool_unpack(pool: int, slot_idx: torch.Tensor, state: torch.Tensor, stream=None) -> None:
-    _cuda(slot_idx, torch.int32, "slot_idx")
-    _cuda(state, torch.float32, "state")
+    """Reconstruct FP32 states [n][H][d_k][d_v] of the slots slot_idx [n]."""
+    _codec_args(pool, slot_idx, state, stream, "damp_pool_unpack")
     _check(_lib.damp_pool_unpack(pool, slot_idx.numel(), _ptr(slot_idx), _ptr(state),
                                  _stream(stream, state.device)), "damp_pool_unpack")
 
 
-def damp_decode_step(pool: int, slot_idx: torch.Tensor, q: torch.Tensor, k: torch.Tensor,
-                     v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
-                     stream=None) -> None:
-    """One decode step.  q, k [n][H][d_k] and v [n][H][d_v] in bf16 or fp32;
-    alpha fp32 [n][H] (GDN) or [n][H][d_k] (KDA); beta fp32 [n][H]; out fp32
-    [n][H][d_v]."""
+def _step_args(pool, slot_idx, q, k, v, alpha, beta, out, stream):
+    """Check every tensor against the pool's (H, d_k, d_v) and the batch size
+    n = slot_idx.numel() before anything is enqueued; returns (dtype, gate)."""
+    _, _, H, d_k, d_v = _pool_shape(pool)
+    if not isinstance(slot_idx, torch.Tensor) or slot_idx.dim() != 1:
+        raise ValueError("slot_idx must be a 1-D tensor")
+    n = slot_idx.numel()
+    _shape(q, "q", (n, H, d_k))
+    _shape(k, "k", (n, H, d_k))
+    _shape(v, "v", (n, H, d_v))
+    _shape(beta, "beta", (n, H))
+    _shape(out, "out", (n, H, d_v))
+    if tuple(alpha.shape) == (n, H, d_k) and alpha.dim() == 3:
+        gate = DAMP_GATE_VECTOR
+    elif tuple(alpha.shape) == (n, H):
+        gate = DAMP_GATE_SCALAR
+    else:
+        raise ValueError(f"alpha must have shape {(n, H)} (GDN) or {(n, H, d_k)} (KDA), "
+                         f"got {tuple(alpha.shape)}")
     _cuda(slot_idx, torch.int32, "slot_idx")
     _cuda(q, None, "q")
     if q.dtype == torch.bfloat16:
@@ -279,10 +349,38 @@ def damp_decode_step(pool: int, slot_idx: torch.Tensor, q: torch.Tensor, k: torc
     _cuda(alpha, torch.float32, "alpha")
     _cuda(beta, torch.float32, "beta")
     _cuda(out, torch.float32, "out")
-    gate = DAMP_GATE_VECTOR if alpha.dim() == 3 else DAMP_GATE_SCALAR
+    _same_device(stream, slot_idx, q, k, v, alpha, beta, out)
+    return dt, gate
+
+
+def damp_decode_step(pool: int, slot_idx: torch.Tensor, q: torch.Tensor, k: torch.Tensor,
+                     v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
+                     stream=None) -> None:
+    """One decode step.  q, k [n][H][d_k] and v [n][H][d_v] in bf16 or fp32;
+    alpha fp32 [n][H] (GDN) or [n][H][d_k] (KDA); beta fp32 [n][H]; out fp32
+    [n][H][d_v]; n = slot_idx.numel()."""
+    dt, gate = _step_args(pool, slot_idx, q, k, v, alpha, beta, out, stream)
     _check(_lib.damp_decode_step(pool, slot_idx.numel(), _ptr(slot_idx), dt, _ptr(q), _ptr(k),
                                  _ptr(v), gate, _ptr(alpha), _ptr(beta), _ptr(out),
                                  _stream(stream, q.device)), "damp_decode_step")
+
+
+def damp_decode_step_validated(pool: int, slot_idx: torch.Tensor, q: torch.Tensor,
+                               k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                               beta: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """damp_decode_step that skips (and flags with DAMP_EFLAG_NONFINITE) every
+    unit whose inputs hold a NaN or an infinity."""
+    dt, gate = _step_args(pool, slot_idx, q, k, v, alpha, beta, out, stream)
+    _check(_lib.damp_decode_step_validated(pool, slot_idx.numel(), _ptr(slot_idx), dt, _ptr(q),
+                                           _ptr(k), _ptr(v), gate, _ptr(alpha), _ptr(beta),
+                                           _ptr(out), _stream(stream, q.device)),
+           "damp_decode_step_validated")
+
+
+def damp_set_test_hooks(wait_limit_ns: int = 0, hooks: int = 0) -> None:
+    """Test hooks of the failure path (process-wide): the bound of the decode
+    step's internal waits (0 = default, 2 s) and DAMP_HOOK_HOLD_FIRST_ITEM."""
+    _check(_lib.damp_set_test_hooks(int(wait_limit_ns), int(hooks)), "damp_set_test_hooks")
 
 
 def damp_validate_slots(slot_idx, n_slots: int) -> None:
@@ -319,10 +417,23 @@ def calib_acc(H: int, d_k: int, device="cuda") -> torch.Tensor:
 def damp_calib_accumulate(pool: int, slot_idx: torch.Tensor, alpha: torch.Tensor,
                           acc: torch.Tensor, stream=None) -> None:
     """Add one step's records of an FP32 pool (states after the step)."""
+    fmt, _, H, d_k, _ = _pool_shape(pool)
+    if fmt != DAMP_FMT_FP32:
+        raise ValueError("damp_calib_accumulate records an FP32 pool")
+    if not isinstance(slot_idx, torch.Tensor) or slot_idx.dim() != 1:
+        raise ValueError("slot_idx must be a 1-D tensor")
+    n = slot_idx.numel()
+    if tuple(alpha.shape) == (n, H, d_k) and alpha.dim() == 3:
+        gate = DAMP_GATE_VECTOR
+    elif tuple(alpha.shape) == (n, H):
+        gate = DAMP_GATE_SCALAR
+    else:
+        raise ValueError(f"alpha must have shape {(n, H)} or {(n, H, d_k)}")
+    _shape(acc, "acc", (damp_calib_bytes(H, d_k) // 8,))
     _cuda(slot_idx, torch.int32, "slot_idx")
     _cuda(alpha, torch.float32, "alpha")
     _cuda(acc, torch.float64, "acc")
-    gate = DAMP_GATE_VECTOR if alpha.dim() == 3 else DAMP_GATE_SCALAR
+    _same_device(stream, slot_idx, alpha, acc)
     _check(_lib.damp_calib_accumulate(pool, slot_idx.numel(), _ptr(slot_idx), gate, _ptr(alpha),
                                       _ptr(acc), _stream(stream, acc.device)),
            "damp_calib_accumulate")
@@ -390,24 +501,25 @@ class DampPool:
     head."""
 
     def __init__(self, fmt, n_slots: int, H: int, d: int, hp_row_idx=None,
-                 device="cuda", fp16_map=None):
+                 device="cuda", fp16_map=None, d_v: int | None = None):
         self.fmt = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
-        self.n_slots, self.H, self.d = n_slots, H, d
+        d_v = d if d_v is None else d_v
+        self.n_slots, self.H, self.d, self.d_k, self.d_v = n_slots, H, d, d, d_v
         if fp16_map is not None:
             if self.fmt != DAMP_FMT_MIXED:
                 raise ValueError("an FP16-row map needs the mixed format")
             fp16_map = np.ascontiguousarray(fp16_map, np.uint8).reshape(H, d)
-            self.nbytes = damp_pool_bytes_map(n_slots, H, d, d, fp16_map)
+            self.nbytes = damp_pool_bytes_map(n_slots, H, d, d_v, fp16_map)
             self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
-            self.handle = damp_pool_create_map(n_slots, H, d, d, fp16_map, self.buf)
+            self.handle = damp_pool_create_map(n_slots, H, d, d_v, fp16_map, self.buf)
             counts = fp16_map.sum(axis=1)
             self.hp = int(counts[0]) if (counts == counts[0]).all() else -1
         else:
             hp_row_idx = None if hp_row_idx is None else np.asarray(hp_row_idx).reshape(H, -1)
             self.hp = 0 if hp_row_idx is None else hp_row_idx.shape[1]
-            self.nbytes = damp_pool_bytes(self.fmt, n_slots, H, d, d, self.hp)
+            self.nbytes = damp_pool_bytes(self.fmt, n_slots, H, d, d_v, self.hp)
             self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
-            self.handle = damp_pool_create(self.fmt, n_slots, H, d, d, self.hp, hp_row_idx,
+            self.handle = damp_pool_create(self.fmt, n_slots, H, d, d_v, self.hp, hp_row_idx,
                                            self.buf)
         self.header_bytes = damp_pool_block_offset(self.handle, 0, 0)
         self.heads = [damp_pool_head_layout(self.handle, h) for h in range(H)]
@@ -450,12 +562,16 @@ class DampPool:
     def unpack(self, slot_idx, state, stream=None):
         damp_pool_unpack(self.handle, slot_idx, state, stream)
 
-    def step(self, slot_idx, q, k, v, alpha, beta, out, stream=None, validate=False):
+    def step(self, slot_idx, q, k, v, alpha, beta, out, stream=None, validate=False,
+             check_inputs=False):
         """One decode step; ``validate`` first checks the slot indices on the
-        host (a device-to-host copy: for debugging, not the serving path)."""
+        host (a device-to-host copy: for debugging, not the serving path);
+        ``check_inputs`` skips and flags units with non-finite inputs on the
+        device (damp_decode_step_validated)."""
         if validate:
             damp_validate_slots(slot_idx, self.n_slots)
-        damp_decode_step(self.handle, slot_idx, q, k, v, alpha, beta, out, stream)
+        f = damp_decode_step_validated if check_inputs else damp_decode_step
+        f(self.handle, slot_idx, q, k, v, alpha, beta, out, stream)
 
     def get_error(self, clear=False, stream=None) -> int:
         return damp_pool_get_error(self.handle, clear, stream, self.buf.device)
@@ -468,7 +584,8 @@ class DampPool:
         for i in range(len(slots)):
             for h in range(self.H):
                 _, st, off = self.heads[h]
-                lg = damp_block_to_logical(self.handle, h, raw[i, off:off + st], self.fmt, self.d)
+                lg = damp_block_to_logical(self.handle, h, raw[i, off:off + st], self.fmt,
+                                           self.d_k, self.d_v)
                 if out is None:
                     out = {k: np.empty((len(slots), self.H) + v.shape, v.dtype)
                            for k, v in lg.items()}

@@ -22,8 +22,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdamp.so")
-SOURCES = ["damp_abi.cu", "damp_decode.cu", "damp_decode_unit.cu", "damp_codec.cu",
-           "damp_calib.cu"]
+SOURCES = ["damp_abi.cu", "damp_decode.cu", "damp_decode_unit.cu", "damp_decode_any.cu",
+           "damp_codec.cu", "damp_calib.cu"]
 HEADERS = ["damp_internal.h", "damp_device.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <atomic>
 #include <chrono>
 #include <new>
 #include <thread>
@@ -21,53 +22,6 @@ struct damp_pool {
     PoolDesc d;
 };
 
-namespace damp {
-
-// Minimum-cost perfect matching of a head's 16 row groups, the cost of a pair
-// being the number of row positions where the two groups differ in format.
-// Exact, by dynamic programming over subsets of groups: the lowest group of a
-// subset is matched first, ties going to its lowest partner.  The pairs are
-// listed in ascending order of their lower group.
-void row_group_order(const uint32_t* mask, uint8_t order[16]) {
-    constexpr int G = 16;
-    uint8_t m[G];
-    bool same = true;
-    for (int g = 0; g < G; ++g) {
-        m[g] = (uint8_t)(mask[g >> 2] >> (8 * (g & 3)));
-        same = same && m[g] == m[0];
-    }
-    if (same) {   // every pairing costs 0: the groups in order (what the search returns)
-        for (int g = 0; g < G; ++g) order[g] = (uint8_t)g;
-        return;
-    }
-    std::vector<uint8_t> cost(1u << G, 0), pick(1u << G, 0);
-    for (uint32_t S = 1; S < (1u << G); ++S) {
-        if (__builtin_popcount(S) & 1) continue;
-        const int i = __builtin_ctz(S);
-        const uint32_t R = S & ~(1u << i);
-        int best = 1 << 30, bj = 0;
-        for (uint32_t T = R; T; T &= T - 1) {
-            const int j = __builtin_ctz(T);
-            const int c = __builtin_popcount((unsigned)(m[i] ^ m[j])) + cost[R & ~(1u << j)];
-            if (c < best) {
-                best = c;
-                bj = j;
-            }
-        }
-        cost[S] = (uint8_t)best;
-        pick[S] = (uint8_t)bj;
-    }
-    uint32_t S = (1u << G) - 1;
-    for (int k = 0; S; ++k) {
-        const int i = __builtin_ctz(S);
-        const int j = pick[S];
-        order[2 * k] = (uint8_t)i;
-        order[2 * k + 1] = (uint8_t)j;
-        S &= ~((1u << i) | (1u << j));
-    }
-}
-
-}  // namespace damp
 
 namespace {
 
@@ -75,35 +29,36 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool dim_ok(int d) { return d >= 16 && d <= damp::kMaxDim && d % 16 == 0; }
+
 int check_shape(int format, int d_k, int d_v, int hp_rows) {
     if (format != DAMP_FMT_FP32 && format != DAMP_FMT_INT8_ROW && format != DAMP_FMT_MIXED &&
         format != DAMP_FMT_FP8_ROW)
         return DAMP_ERR_INVALID_ARGUMENT;
+    if (!dim_ok(d_k) || !dim_ok(d_v)) return DAMP_ERR_UNSUPPORTED;
     if (hp_rows < 0 || hp_rows > d_k) return DAMP_ERR_INVALID_ARGUMENT;
     if (format != DAMP_FMT_MIXED && hp_rows != 0) return DAMP_ERR_INVALID_ARGUMENT;
-    if (d_k != d_v) return DAMP_ERR_UNSUPPORTED;
-    if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return DAMP_ERR_UNSUPPORTED;
     return DAMP_OK;
 }
 
-void layout(int format, int d, int hp, size_t* bytes, size_t* stride, uint32_t* f16_off,
-            uint32_t* i8_off) {
+void layout(int format, int d_k, int d_v, int hp, size_t* bytes, size_t* stride,
+            uint32_t* f16_off, uint32_t* i8_off) {
     if (format == DAMP_FMT_FP32) {
-        *bytes = (size_t)d * d * 4;
+        *bytes = (size_t)d_k * d_v * 4;
         *stride = *bytes;
         *f16_off = *i8_off = 0;
         return;
     }
-    const size_t r = (size_t)(d - hp);
-    *bytes = 4 * r + 2 * (size_t)hp * d + r * d;
+    const size_t r = (size_t)(d_k - hp);
+    *bytes = 4 * r + 2 * (size_t)hp * d_v + r * d_v;
     const size_t scales = align_up(4 * r, 16);
     *f16_off = (uint32_t)scales;
-    *i8_off = (uint32_t)(scales + 2 * (size_t)hp * d);
-    *stride = align_up(scales + 2 * (size_t)hp * d + r * d, 16);
+    *i8_off = (uint32_t)(scales + 2 * (size_t)hp * d_v);
+    *stride = align_up(scales + 2 * (size_t)hp * d_v + r * d_v, 16);
 }
 
-size_t header_bytes(int H) {
-    return align_up(damp::head_table_offset(H) + (size_t)H * 16, 256);
+size_t header_bytes(int H, int d_k) {
+    return align_up(damp::head_table_offset(H, d_k) + (size_t)H * 16, 256);
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? DAMP_OK : DAMP_ERR_CUDA; }
@@ -120,7 +75,8 @@ const char* damp_status_string(int status) {
     switch (status) {
         case DAMP_OK: return "ok";
         case DAMP_ERR_INVALID_ARGUMENT: return "invalid argument";
-        case DAMP_ERR_UNSUPPORTED: return "unsupported shape (d_k == d_v in {16, 32, 64, 128})";
+        case DAMP_ERR_UNSUPPORTED:
+            return "unsupported shape (d_k, d_v multiples of 16 in [16, 256])";
         case DAMP_ERR_MISALIGNED: return "pointer not 16-byte aligned";
         case DAMP_ERR_BUFFER_TOO_SMALL: return "pool buffer too small";
         case DAMP_ERR_CUDA: return "CUDA runtime error";
@@ -135,7 +91,7 @@ int damp_layout(int format, int d_k, int d_v, int hp_rows, size_t* block_bytes,
     if (rc) return rc;
     size_t b, s;
     uint32_t f, i;
-    layout(format, d_k, hp_rows, &b, &s, &f, &i);
+    layout(format, d_k, d_v, hp_rows, &b, &s, &f, &i);
     if (block_bytes) *block_bytes = b;
     if (block_stride) *block_stride = s;
     return DAMP_OK;
@@ -153,7 +109,7 @@ struct Layout {
     size_t slot_stride = 0, max_bytes = 0, max_stride = 0;
 };
 
-Layout pool_layout(int format, int H, int d, const std::vector<uint32_t>& masks) {
+Layout pool_layout(int format, int H, int d_k, int d_v, const std::vector<uint32_t>& masks) {
     Layout L;
     L.heads.assign((size_t)H * 4, 0u);
     for (int h = 0; h < H; ++h) {
@@ -162,7 +118,7 @@ Layout pool_layout(int format, int H, int d, const std::vector<uint32_t>& masks)
             hp += __builtin_popcount(masks[(size_t)h * damp::kMaskWords + w]);
         size_t b, st;
         uint32_t f16, i8;
-        layout(format, d, hp, &b, &st, &f16, &i8);
+        layout(format, d_k, d_v, hp, &b, &st, &f16, &i8);
         uint32_t* e = &L.heads[(size_t)h * 4];
         e[0] = (uint32_t)L.slot_stride;
         e[1] = (uint32_t)st;
@@ -186,8 +142,8 @@ int damp_pool_bytes(int format, int n_slots, int H, int d_k, int d_v, int hp_row
     if (rc) return rc;
     size_t b, s;
     uint32_t f, i;
-    layout(format, d_k, hp_rows, &b, &s, &f, &i);
-    *bytes = header_bytes(H) + (size_t)n_slots * H * s;
+    layout(format, d_k, d_v, hp_rows, &b, &s, &f, &i);
+    *bytes = header_bytes(H, d_k) + (size_t)n_slots * H * s;
     return DAMP_OK;
 }
 
@@ -207,23 +163,24 @@ int masks_from_map(int H, int d_k, const uint8_t* is_fp16, std::vector<uint32_t>
     return DAMP_OK;
 }
 
-int create_common(int format, int n_slots, int H, int d_k, int hp_rows,
+int create_common(int format, int n_slots, int H, int d_k, int d_v, int hp_rows,
                   const std::vector<uint32_t>& masks, void* dev_buf, size_t buf_bytes,
                   damp_pool** out) {
-    const Layout L = pool_layout(format, H, d_k, masks);
+    const Layout L = pool_layout(format, H, d_k, d_v, masks);
     if (L.slot_stride > 0xffffffffull) return DAMP_ERR_UNSUPPORTED;
     PoolDesc d{};
     d.format = format;
     d.n_slots = n_slots;
     d.H = H;
-    d.d = d_k;
+    d.d_k = d_k;
+    d.d_v = d_v;
     d.hp = hp_rows;
     d.block_bytes = L.max_bytes;
     d.block_stride = L.max_stride;
     d.slot_stride = L.slot_stride;
-    d.header_bytes = header_bytes(H);
+    d.header_bytes = header_bytes(H, d_k);
     d.dir_off = damp::dir_offset(H);
-    d.head_off = damp::head_table_offset(H);
+    d.head_off = damp::head_table_offset(H, d_k);
     d.pool_bytes = d.header_bytes + (size_t)n_slots * d.slot_stride;
     if (dev_buf) {
         if (!aligned16(dev_buf)) return DAMP_ERR_MISALIGNED;
@@ -258,17 +215,14 @@ int create_common(int format, int n_slots, int H, int d_k, int hp_rows,
                     const bool f16 = (masks[(size_t)h * damp::kMaskWords + (i >> 5)] >> (i & 31)) & 1u;
                     uint32_t e;
                     if (f16) {
-                        e = (f16_off + r16 * 2u * d_k) | (1u << 31);
+                        e = damp::dir_entry(f16_off + r16 * 2u * (uint32_t)d_v, 0u, true);
                         ++r16;
                     } else {
-                        e = (i8_off + r8 * (uint32_t)d_k) | ((4u * r8) << 16);
+                        e = damp::dir_entry(i8_off + r8 * (uint32_t)d_v, 4u * r8, false);
                         ++r8;
                     }
-                    dir[(size_t)h * damp::kDirStride + i] = e;
+                    dir[(size_t)h * d_k + i] = e;
                 }
-                damp::row_group_order(masks.data() + (size_t)h * damp::kMaskWords,
-                                      reinterpret_cast<uint8_t*>(dir + (size_t)h * damp::kDirStride +
-                                                                 damp::kDirWords));
             }
         }
         cudaError_t e = cudaMemcpy(dev_buf, hdr.data(), hdr.size(), cudaMemcpyHostToDevice);
@@ -306,7 +260,7 @@ int damp_pool_create(int format, int n_slots, int H, int d_k, int d_v, int hp_ro
             if (w & (1u << (i & 31))) return DAMP_ERR_INVALID_ARGUMENT;  // repeated row
             w |= 1u << (i & 31);
         }
-    return create_common(format, n_slots, H, d_k, hp_rows, masks, dev_buf, buf_bytes, out);
+    return create_common(format, n_slots, H, d_k, d_v, hp_rows, masks, dev_buf, buf_bytes, out);
 }
 
 int damp_pool_bytes_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is_fp16,
@@ -316,8 +270,8 @@ int damp_pool_bytes_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is_
     if (rc) return rc;
     std::vector<uint32_t> masks;
     if ((rc = masks_from_map(H, d_k, is_fp16, &masks))) return rc;
-    const Layout L = pool_layout(DAMP_FMT_MIXED, H, d_k, masks);
-    *bytes = header_bytes(H) + (size_t)n_slots * L.slot_stride;
+    const Layout L = pool_layout(DAMP_FMT_MIXED, H, d_k, d_v, masks);
+    *bytes = header_bytes(H, d_k) + (size_t)n_slots * L.slot_stride;
     return DAMP_OK;
 }
 
@@ -338,14 +292,8 @@ int damp_pool_create_map(int n_slots, int H, int d_k, int d_v, const uint8_t* is
             c += __builtin_popcount(masks[(size_t)h * damp::kMaskWords + w]);
         hp = (h == 0 || c == hp) ? c : -2;
     }
-    return create_common(DAMP_FMT_MIXED, n_slots, H, d_k, hp < 0 ? -1 : hp, masks, dev_buf,
+    return create_common(DAMP_FMT_MIXED, n_slots, H, d_k, d_v, hp < 0 ? -1 : hp, masks, dev_buf,
                          buf_bytes, out);
-}
-
-int damp_pool_row_groups(const damp_pool* pool, int h, uint8_t* order) {
-    if (!pool || !order || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
-    damp::row_group_order(pool->d.host_masks + (size_t)h * damp::kMaskWords, order);
-    return DAMP_OK;
 }
 
 int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,
@@ -355,11 +303,11 @@ int damp_pool_head_layout(const damp_pool* pool, int h, size_t* block_bytes,
     const uint32_t* e = d.host_heads + (size_t)h * 4;
     if (block_bytes) {
         if (d.format == DAMP_FMT_FP32) {
-            *block_bytes = (size_t)d.d * d.d * 4;
+            *block_bytes = (size_t)d.d_k * d.d_v * 4;
         } else {
-            const size_t r = (size_t)(e[3] - e[2]) / (2 * (size_t)d.d);   // FP16 rows
-            const size_t r8 = (size_t)d.d - r;
-            *block_bytes = 4 * r8 + 2 * r * d.d + r8 * d.d;
+            const size_t r = (size_t)(e[3] - e[2]) / (2 * (size_t)d.d_v);   // FP16 rows
+            const size_t r8 = (size_t)d.d_k - r;
+            *block_bytes = 4 * r8 + 2 * r * d.d_v + r8 * d.d_v;
         }
     }
     if (block_stride) *block_stride = e[1];
@@ -403,8 +351,10 @@ static int codec_args(const damp_pool* pool, int n, const int32_t* slot_idx, con
     a->n_slots = d.n_slots;
     a->heads = reinterpret_cast<const uint4*>(d.dev_buf + d.head_off);
     a->slot_stride = d.slot_stride;
-    const int upi = 128 / d.d;
-    a->n_items = (int)(((size_t)n * d.H + upi - 1) / upi);
+    a->d_k = d.d_k;
+    a->d_v = d.d_v;
+    a->format = d.format;
+    a->n_items = n * d.H;   // units (the launcher groups them)
     return DAMP_OK;
 }
 
@@ -424,9 +374,17 @@ int damp_pool_unpack(const damp_pool* pool, int n, const int32_t* slot_idx, floa
     return cuda_status(damp::launch_unpack(pool->d, a, static_cast<cudaStream_t>(stream)));
 }
 
-int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int in_dtype,
-                     const void* q, const void* k, const void* v, int gate, const float* alpha,
-                     const float* beta, float* out, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Test hooks of the failure path (damp_set_test_hooks).
+std::atomic<unsigned long long> g_wait_ns{0};
+std::atomic<uint32_t> g_hooks{0};
+
+int decode_common(const damp_pool* pool, int n, const int32_t* slot_idx, int in_dtype,
+                  const void* q, const void* k, const void* v, int gate, const float* alpha,
+                  const float* beta, float* out, void* stream, int validate) {
     if (!pool || n < 0) return DAMP_ERR_INVALID_ARGUMENT;
     const PoolDesc& d = pool->d;
     if (!d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
@@ -442,6 +400,9 @@ int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int 
         return DAMP_ERR_MISALIGNED;
     if ((size_t)n * d.H > (size_t)0x7fffffff) return DAMP_ERR_UNSUPPORTED;
     damp::StepArgs a{};
+    a.d_k = d.d_k;
+    a.d_v = d.d_v;
+    a.format = d.format;
     a.blocks = d.dev_buf + d.header_bytes;
     a.masks = reinterpret_cast<const uint32_t*>(d.dev_buf + damp::kStatusBytes);
     a.dir = reinterpret_cast<const uint32_t*>(d.dev_buf + d.dir_off);
@@ -459,10 +420,37 @@ int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int 
     a.heads = reinterpret_cast<const uint4*>(d.dev_buf + d.head_off);
     a.slot_stride = d.slot_stride;
     a.block_stride = (uint32_t)d.block_stride;
-    const int upi = 128 / d.d;
-    a.n_items = (int)(((size_t)n * d.H + upi - 1) / upi);
+    a.n_items = n * d.H;   // units (the launcher groups them)
+    const unsigned long long wait = g_wait_ns.load(std::memory_order_relaxed);
+    a.wait_ns = wait ? wait : damp::kDefaultWaitNs;
+    a.hooks = g_hooks.load(std::memory_order_relaxed);
+    a.validate = validate;
     return cuda_status(
         damp::launch_decode_step(d, a, in_dtype, gate, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int damp_decode_step(const damp_pool* pool, int n, const int32_t* slot_idx, int in_dtype,
+                     const void* q, const void* k, const void* v, int gate, const float* alpha,
+                     const float* beta, float* out, void* stream) {
+    return decode_common(pool, n, slot_idx, in_dtype, q, k, v, gate, alpha, beta, out, stream, 0);
+}
+
+int damp_decode_step_validated(const damp_pool* pool, int n, const int32_t* slot_idx,
+                               int in_dtype, const void* q, const void* k, const void* v,
+                               int gate, const float* alpha, const float* beta, float* out,
+                               void* stream) {
+    return decode_common(pool, n, slot_idx, in_dtype, q, k, v, gate, alpha, beta, out, stream, 1);
+}
+
+int damp_set_test_hooks(uint64_t wait_limit_ns, uint32_t hooks) {
+    if (hooks & ~DAMP_HOOK_HOLD_FIRST_ITEM) return DAMP_ERR_INVALID_ARGUMENT;
+    g_wait_ns.store(wait_limit_ns, std::memory_order_relaxed);
+    g_hooks.store(hooks, std::memory_order_relaxed);
+    return DAMP_OK;
 }
 
 size_t damp_calib_bytes(int H, int d_k) {
@@ -491,12 +479,14 @@ int damp_calib_accumulate(const damp_pool* pool, int n, const int32_t* slot_idx,
     a.H = d.H;
     a.n_slots = d.n_slots;
     a.gate = gate;
-    return cuda_status(damp::launch_calib_accumulate(a, d.d, static_cast<cudaStream_t>(stream)));
+    a.d_k = d.d_k;
+    a.d_v = d.d_v;
+    return cuda_status(damp::launch_calib_accumulate(a, static_cast<cudaStream_t>(stream)));
 }
 
 static int calib_shape(int H, int d_k) {
     if (H <= 0 || d_k <= 0) return DAMP_ERR_INVALID_ARGUMENT;
-    if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return DAMP_ERR_UNSUPPORTED;
+    if (!dim_ok(d_k)) return DAMP_ERR_UNSUPPORTED;
     return DAMP_OK;
 }
 
@@ -585,25 +575,25 @@ int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float
     if (!pool || !block || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
     const PoolDesc& d = pool->d;
     const uint8_t* b = static_cast<const uint8_t*>(block);
-    const int D = d.d;
+    const int DK = d.d_k, DV = d.d_v;
     if (d.format == DAMP_FMT_FP32) {
         if (!f32) return DAMP_ERR_INVALID_ARGUMENT;
-        memcpy(f32, b, (size_t)D * D * 4);
+        memcpy(f32, b, (size_t)DK * DV * 4);
         return DAMP_OK;
     }
     if (!scale || !half || !code) return DAMP_ERR_INVALID_ARGUMENT;
     const uint32_t f16_off = d.host_heads[(size_t)h * 4 + 2], i8_off = d.host_heads[(size_t)h * 4 + 3];
     int r16 = 0, r8 = 0;
-    for (int i = 0; i < D; ++i) {
+    for (int i = 0; i < DK; ++i) {
         if (is_fp16_row(d, h, i)) {
             scale[i] = 0.0f;
-            memcpy(half + (size_t)i * D, b + f16_off + (size_t)r16 * 2 * D, (size_t)2 * D);
-            memset(code + (size_t)i * D, 0, D);
+            memcpy(half + (size_t)i * DV, b + f16_off + (size_t)r16 * 2 * DV, (size_t)2 * DV);
+            memset(code + (size_t)i * DV, 0, DV);
             ++r16;
         } else {
             memcpy(&scale[i], b + (size_t)r8 * 4, 4);
-            memcpy(code + (size_t)i * D, b + i8_off + (size_t)r8 * D, D);
-            memset(half + (size_t)i * D, 0, (size_t)2 * D);
+            memcpy(code + (size_t)i * DV, b + i8_off + (size_t)r8 * DV, DV);
+            memset(half + (size_t)i * DV, 0, (size_t)2 * DV);
             ++r8;
         }
     }
@@ -616,27 +606,47 @@ int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
     if (!pool || !block || h < 0 || h >= pool->d.H) return DAMP_ERR_INVALID_ARGUMENT;
     const PoolDesc& d = pool->d;
     uint8_t* b = static_cast<uint8_t*>(block);
-    const int D = d.d;
+    const int DK = d.d_k, DV = d.d_v;
     if (d.format == DAMP_FMT_FP32) {
         if (!f32) return DAMP_ERR_INVALID_ARGUMENT;
-        memcpy(b, f32, (size_t)D * D * 4);
+        memcpy(b, f32, (size_t)DK * DV * 4);
         return DAMP_OK;
     }
     if (!scale || !half || !code) return DAMP_ERR_INVALID_ARGUMENT;
     const uint32_t f16_off = d.host_heads[(size_t)h * 4 + 2], i8_off = d.host_heads[(size_t)h * 4 + 3];
     memset(b, 0, d.host_heads[(size_t)h * 4 + 1]);
     int r16 = 0, r8 = 0;
-    for (int i = 0; i < D; ++i) {
+    for (int i = 0; i < DK; ++i) {
         if (is_fp16_row(d, h, i)) {
-            memcpy(b + f16_off + (size_t)r16 * 2 * D, half + (size_t)i * D, (size_t)2 * D);
+            memcpy(b + f16_off + (size_t)r16 * 2 * DV, half + (size_t)i * DV, (size_t)2 * DV);
             ++r16;
         } else {
             memcpy(b + (size_t)r8 * 4, &scale[i], 4);
-            memcpy(b + i8_off + (size_t)r8 * D, code + (size_t)i * D, D);
+            memcpy(b + i8_off + (size_t)r8 * DV, code + (size_t)i * DV, DV);
             ++r8;
         }
     }
     return DAMP_OK;
+}
+
+int damp_pool_read_raw(const damp_pool* pool, int slot, int h, void* host_out) {
+    if (!pool || !host_out || !pool->d.dev_buf) return DAMP_ERR_INVALID_ARGUMENT;
+    const PoolDesc& d = pool->d;
+    if (slot < 0 || slot >= d.n_slots || h < 0 || h >= d.H) return DAMP_ERR_INVALID_ARGUMENT;
+    const uint32_t stride = d.host_heads[(size_t)h * 4 + 1];
+    std::vector<uint8_t> raw(stride);
+    const size_t off = d.header_bytes + (size_t)slot * d.slot_stride + d.host_heads[(size_t)h * 4];
+    if (cudaMemcpy(raw.data(), d.dev_buf + off, stride, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return DAMP_ERR_CUDA;
+    const size_t ne = (size_t)d.d_k * d.d_v;
+    uint8_t* o = static_cast<uint8_t*>(host_out);
+    if (d.format == DAMP_FMT_FP32)
+        return damp_block_to_logical(pool, h, raw.data(), nullptr, nullptr, nullptr,
+                                     reinterpret_cast<float*>(o));
+    float* scale = reinterpret_cast<float*>(o);
+    uint16_t* half = reinterpret_cast<uint16_t*>(o + 4 * (size_t)d.d_k);
+    int8_t* code = reinterpret_cast<int8_t*>(o + 4 * (size_t)d.d_k + 2 * ne);
+    return damp_block_to_logical(pool, h, raw.data(), scale, half, code, nullptr);
 }
 
 }  // extern "C"

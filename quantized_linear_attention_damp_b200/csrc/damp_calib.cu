@@ -42,21 +42,22 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
-template <int D>
+// Warp (h, i) owns the totals of key row i of head h; lane l holds columns
+// l + 32t (t < EPL) of the row, zero past d_v (a zero adds no error).
+template <int EPL>
 __global__ void __launch_bounds__(kCalRows * 32)
     calib_accumulate_kernel(CalibArgs a) {
-    constexpr int EPL = D >= 32 ? D / 32 : 1;   // elements per lane
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.x;
+    const int d_k = a.d_k, d_v = a.d_v;
     const int i = blockIdx.y * kCalRows + (threadIdx.x >> 5);
-    if (i >= D) return;
-    const size_t hi = (size_t)h * D + i;
+    if (i >= d_k) return;
+    const size_t hi = (size_t)h * d_k + i;
     double* energy = a.acc;
-    double* retention = a.acc + (size_t)a.H * D;
-    double* count = a.acc + 2 * (size_t)a.H * D;
+    double* retention = a.acc + (size_t)a.H * d_k;
+    double* count = a.acc + 2 * (size_t)a.H * d_k;
     double e_acc = energy[hi], r_acc = retention[hi];
     int cnt = 0;
-    const bool live = D >= 32 || lane < D;
 
     for (int b0 = 0; b0 < a.n; b0 += kCalUnroll) {
         int slot[kCalUnroll];
@@ -66,19 +67,12 @@ __global__ void __launch_bounds__(kCalRows * 32)
             const int b = b0 + u;
             slot[u] = b < a.n ? __ldg(a.slot_idx + b) : -1;
             const bool ok = slot[u] >= 0 && slot[u] < a.n_slots;
-            const float* row = a.state + ((size_t)(ok ? slot[u] : 0) * a.H + h) * D * D +
-                               (size_t)i * D;
-            if constexpr (D == 128) {
-                float4 t = ok ? __ldg(reinterpret_cast<const float4*>(row) + lane)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-                x[u][0] = t.x;
-                x[u][1] = t.y;
-                x[u][2] = t.z;
-                x[u][3] = t.w;
-            } else {
+            const float* row = a.state + ((size_t)(ok ? slot[u] : 0) * a.H + h) * d_k * d_v +
+                               (size_t)i * d_v;
 #pragma unroll
-                for (int t = 0; t < EPL; ++t)
-                    x[u][t] = (ok && live) ? __ldg(row + lane + 32 * t) : 0.0f;
+            for (int t = 0; t < EPL; ++t) {
+                const int j = lane + 32 * t;
+                x[u][t] = (ok && j < d_v) ? __ldg(row + j) : 0.0f;
             }
         }
 #pragma unroll
@@ -97,11 +91,10 @@ __global__ void __launch_bounds__(kCalRows * 32)
             row_scale(m, s, inv);
             double e = 0.0;
 #pragma unroll
-            for (int t = 0; t < EPL; ++t)
-                if (live) e = __dadd_rn(e, lane_error(x[u][t], s, inv));
+            for (int t = 0; t < EPL; ++t) e = __dadd_rn(e, lane_error(x[u][t], s, inv));
             e = warp_sum(e);
             const float al = a.gate == DAMP_GATE_VECTOR
-                                 ? __ldg(a.alpha + ((size_t)b * a.H + h) * D + i)
+                                 ? __ldg(a.alpha + ((size_t)b * a.H + h) * d_k + i)
                                  : __ldg(a.alpha + (size_t)b * a.H + h);
             e_acc = __dadd_rn(e_acc, e);
             r_acc = __dadd_rn(r_acc, __dmul_rn((double)al, (double)al));
@@ -127,11 +120,11 @@ __device__ __forceinline__ double calib_score(const double* acc, int H, int D, i
 
 // One CTA per head, one thread per key row: rank by counting (ties to the
 // lower row), then the selected rows' positions by a prefix count.
-__global__ void __launch_bounds__(kMaxD)
+__global__ void __launch_bounds__(kMaxDim)
     calib_select_kernel(const double* acc, int H, int D, int hp, double* score,
                         uint16_t* idx) {
-    __shared__ double sc[kMaxD];
-    __shared__ int sel[kMaxD];
+    __shared__ double sc[kMaxDim];
+    __shared__ int sel[kMaxDim];
     const int h = blockIdx.x, i = threadIdx.x;
     const double s = i < D ? calib_score(acc, H, D, h, i) : 0.0;
     sc[i] = s;
@@ -192,13 +185,17 @@ __global__ void calib_count_kernel(const uint8_t* is_fp16, int D, int32_t* hp) {
 
 }  // namespace
 
-cudaError_t launch_calib_accumulate(const CalibArgs& a, int d, cudaStream_t stream) {
-    const dim3 grid(a.H, (d + kCalRows - 1) / kCalRows);
-    switch (d) {
-        case 16: calib_accumulate_kernel<16><<<grid, kCalRows * 32, 0, stream>>>(a); break;
-        case 32: calib_accumulate_kernel<32><<<grid, kCalRows * 32, 0, stream>>>(a); break;
-        case 64: calib_accumulate_kernel<64><<<grid, kCalRows * 32, 0, stream>>>(a); break;
-        case 128: calib_accumulate_kernel<128><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+cudaError_t launch_calib_accumulate(const CalibArgs& a, cudaStream_t stream) {
+    const dim3 grid(a.H, (a.d_k + kCalRows - 1) / kCalRows);
+    switch ((a.d_v + 31) / 32) {
+        case 1: calib_accumulate_kernel<1><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 2: calib_accumulate_kernel<2><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 3: calib_accumulate_kernel<3><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 4: calib_accumulate_kernel<4><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 5: calib_accumulate_kernel<5><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 6: calib_accumulate_kernel<6><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 7: calib_accumulate_kernel<7><<<grid, kCalRows * 32, 0, stream>>>(a); break;
+        case 8: calib_accumulate_kernel<8><<<grid, kCalRows * 32, 0, stream>>>(a); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -206,7 +203,7 @@ cudaError_t launch_calib_accumulate(const CalibArgs& a, int d, cudaStream_t stre
 
 cudaError_t launch_calib_select(const double* acc, int H, int d, int hp, double* score,
                                 uint16_t* idx, cudaStream_t stream) {
-    calib_select_kernel<<<H, kMaxD, 0, stream>>>(acc, H, d, hp, score, idx);
+    calib_select_kernel<<<H, kMaxDim, 0, stream>>>(acc, H, d, hp, score, idx);
     return cudaGetLastError();
 }
 
@@ -264,7 +261,7 @@ extern "C" int damp_calib_select_budget_static(int H, int d_k, int budget, const
                                                uint8_t* is_fp16, int32_t* hp_per_head,
                                                void* stream) {
     if (H <= 0 || d_k <= 0) return DAMP_ERR_INVALID_ARGUMENT;
-    if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return DAMP_ERR_UNSUPPORTED;
+    if (d_k < 16 || d_k > damp::kMaxDim || d_k % 16) return DAMP_ERR_UNSUPPORTED;
     if ((size_t)H * d_k > (size_t)damp::kStaticScores) return DAMP_ERR_UNSUPPORTED;
     if (budget < 0 || budget > H * d_k || !acc || !is_fp16 || !hp_per_head)
         return DAMP_ERR_INVALID_ARGUMENT;

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
         uint32_t bits = 0;
         int rank16 = 0;
         if (QUANT && ok) {
-            const uint4 mw = __ldg(reinterpret_cast<const uint4*>(a.masks) + h);
+            const uint4 mw = __ldg(reinterpret_cast<const uint4*>(a.masks + (size_t)h * kMaskWords));
             row_formats<D>(mw, r0, bits, rank16);
         }
         float2 x[RPT][2];
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
                 continue;
             }
             if constexpr (QUANT) {
-                load_tile_gdir<D, FP8>(blk, a.dir + (size_t)h * kDirStride, r0, cg, x);
+                load_tile_gdir<D, FP8>(blk, a.dir + (size_t)h * D, r0, cg, x);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {
@@ -116,9 +116,17 @@ cudaError_t dispatch_d(int format, const CodecArgs& a, cudaStream_t s) {
     return launch_codec_t<D, true, PACK, false>(a, s);
 }
 
+// Square d in {16, 32, 64, 128}: the thread-tile kernel above (a.n_items
+// counts units; an item holds 128/d of them); any other shape: the one-CTA-
+// per-unit kernels of damp_decode_any.cu.
 template <bool PACK>
-cudaError_t dispatch(const PoolDesc& p, const CodecArgs& a, cudaStream_t s) {
-    switch (p.d) {
+cudaError_t dispatch(const PoolDesc& p, const CodecArgs& a0, cudaStream_t s) {
+    CodecArgs a = a0;
+    if (p.d_k != p.d_v || p.d_k > kMaxFastD || (p.d_k & (p.d_k - 1)))
+        return PACK ? launch_pack_any(a, s) : launch_unpack_any(a, s);
+    const int upi = kMaxFastD / p.d_k;
+    a.n_items = (a.n_items + upi - 1) / upi;
+    switch (p.d_k) {
         case 16: return dispatch_d<16, PACK>(p.format, a, s);
         case 32: return dispatch_d<32, PACK>(p.format, a, s);
         case 64: return dispatch_d<64, PACK>(p.format, a, s);

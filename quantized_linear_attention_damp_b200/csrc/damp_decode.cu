@@ -135,12 +135,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         }
         const uint32_t tx_all = __reduce_add_sync(0xffffffffu, tx);
         __syncwarp();
-        if (lane == 0) {
+        const bool hold = il == 0 && (a.hooks & kHookHoldFirstItem);
+        if (lane == 0 && !hold) {
             if (tx_all) mbar_arrive_expect_tx(full_bar(stage), tx_all);
             else mbar_arrive(full_bar(stage));
         }
         __syncwarp();
-        if (load) {
+        if (load && !hold) {
             const int item = (int)blockIdx.x + il * (int)gridDim.x;
             const int u = item * UPI + lane;
             const int h = u % a.H;
@@ -158,8 +159,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
                 bulk_g2s(smem_u32(st + a.st_alpha + lane * D * 4), a.alpha + (size_t)u * D, D * 4,
                          fb);
             if constexpr (QUANT)
-                bulk_g2s(smem_u32(st + a.st_dir + lane * D * 4), a.dir + (size_t)h * kDirStride,
-                         D * 4, fb);
+                bulk_g2s(smem_u32(st + a.st_dir + lane * D * 4), a.dir + (size_t)h * D, D * 4,
+                         fb);
         }
     };
 
@@ -184,8 +185,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
     };
 
     const int ahead = NS - 2;
+    int issued = 0;   // items issued so far (meaningful in the issue warp)
     if (warp == kIssueWarp)
-        for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
+        for (; issued < ahead && issued < my_items; ++issued) issue(issued);
 
     // ---- consumer side (all 8 warps)
     const int ui = tid / G::TPU;        // unit within the item
@@ -200,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
     float* delta_s = red_w + UPI * 8 * D;                              // [UPI][D]
     float* cpart_s = delta_s + UPI * D;                                // [UPI][8]
     float* rowbuf = cpart_s + UPI * 8 + (ui * 8 + rg) * 2 * RPT;       // this row group's
+    int* s_bad = reinterpret_cast<int*>(cpart_s + UPI * 8 + 16 * UPI * RPT);   // [UPI] (a.validate)
 
     int it = 0;
     bool aborted = false;
@@ -207,9 +210,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         const int item = (int)blockIdx.x + it * (int)gridDim.x;
         const int stage = it % NS;
         const uint32_t parity = static_cast<uint32_t>(it / NS) & 1u;
-        const bool ok = mbar_wait_bounded(full_bar(stage), parity);
+        // a warp whose wait gave up in any lane skips the item; the CTA leaves
+        // the loop together at the first barrier below
+        const bool ok =
+            __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(stage), parity, a.wait_ns));
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
         const Meta meta = *reinterpret_cast<const Meta*>(st + a.st_meta + ui * sizeof(Meta));
+        if (tid < UPI) s_bad[tid] = 0;
         const int u = item * UPI + ui;
         const bool active = ok && meta.exists && meta.slot >= 0 && meta.slot < a.n_slots;
         uint8_t* blk = st + ui * a.block_stride;
@@ -303,11 +310,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             aborted = true;
             break;
         }
-        if (warp == kIssueWarp && it + ahead < my_items) issue(it + ahead);
+        if (warp == kIssueWarp && it + ahead < my_items) {
+            issue(it + ahead);
+            issued = it + ahead + 1;
+        }
 
         // ---- step 2 (second half) + step 3: per column j, delta_j and out_j
         if (tu < D) {
             const int j = tu;
+            if (active && a.validate) {
+                const float aj = KDA ? salpha[j] : meta.alpha;
+                if (!(isfinite(load_in<BF16>(sq, j)) && isfinite(load_in<BF16>(sk, j)) &&
+                      isfinite(load_in<BF16>(st + a.st_v + ui * D * ELT, j)) && isfinite(aj) &&
+                      isfinite(meta.beta)))
+                    atomicOr(&s_bad[ui], 1);
+            }
             if (active) {
                 const float* cu = red_u + ui * 8 * D + j;
                 const float* cw = red_w + ui * 8 * D + j;
@@ -331,9 +348,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
             }
         }
         __syncthreads();
+        if (active && s_bad[ui]) {
+            // a non-finite input: the unit is skipped (out row zeroed, block
+            // neither updated nor stored)
+            if (tu < D) a.out[(size_t)u * D + tu] = 0.f;
+            if (tu == 0) {
+                reinterpret_cast<Meta*>(st + a.st_meta + ui * sizeof(Meta))->slot = -1;
+                atomicOr(a.status, DAMP_EFLAG_NONFINITE);
+            }
+        }
 
         // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
-        if (active) {
+        if (active && !s_bad[ui]) {
             const float4 dl = *reinterpret_cast<const float4*>(delta_s + ui * D + 4 * cg);
             const float2 d0 = make_float2(dl.x, dl.y), d1 = make_float2(dl.z, dl.w);
 #pragma unroll
@@ -360,19 +386,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const StepArgs
         if (tid == 0) store_item(it);
     }
 
-    if (tid == 0) {
-        if (aborted) {
-            atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
-            // drain loads that may still be landing in this CTA's stages
-            for (int j = 0; j <= ahead; ++j) {
-                const int jt = it + j;
-                if (jt >= my_items) break;
-                (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
-                                        100000000ull);
-            }
-        }
-        bulk_wait_all<0>();
+    if (aborted && warp == kIssueWarp && lane == 0) {
+        atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
+        // loads still landing in this CTA's stages: the items the issue warp
+        // issued after the last one consumed (it .. issued-1)
+        for (int jt = it; jt < issued; ++jt)
+            (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
+                                    100000000ull);
     }
+    if (tid == 0) bulk_wait_all<0>();
 }
 
 // ---------------------------------------------------------------------- host
@@ -402,8 +424,9 @@ Layout stage_layout(int d, uint32_t stride, int in_dtype, int gate) {
     L.st_meta = off;
     off += upi * sizeof(Meta);
     L.stage_bytes = align_up(off, 128);
-    // red_u + red_w [128/d][8][d] each, delta [128], cpart [8*128/d], rowbuf 2*128
-    L.scratch_bytes = align_up((2 * 8 * 128 + 128 + 8 * upi + 2 * 128) * 4, 128);
+    // red_u + red_w [128/d][8][d] each, delta [128], cpart [8*128/d], rowbuf 2*128,
+    // non-finite flags [128/d]
+    L.scratch_bytes = align_up((2 * 8 * 128 + 128 + 8 * upi + 2 * 128 + 8) * 4, 128);
     return L;
 }
 
@@ -523,25 +546,34 @@ cudaError_t prepare_d(int codec) {
 cudaError_t prepare_decode(const PoolDesc& p) {
     const int c = codec_of(p.format);
     cudaError_t e;
-    switch (p.d) {
+    if (p.d_k != p.d_v) return cudaSuccess;   // the one-CTA-per-unit kernel needs no set-up
+    switch (p.d_k) {
         case 16: return prepare_d<16>(c);
         case 32: return prepare_d<32>(c);
         case 64: return prepare_d<64>(c);
         case 128:
             if ((e = prepare_d<128>(c)) != cudaSuccess) return e;
             return c != 0 ? prepare_decode_unit() : cudaSuccess;
-        default: return cudaErrorInvalidValue;
+        default: return cudaSuccess;
     }
 }
 
-cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a, int in_dtype, int gate,
+// Kernel choice.  a.n_items counts units on entry.  d = 128 quantized states:
+// the row-pair kernel (damp_decode_unit.cu) whenever three stages of a block
+// fit in shared memory; square d in {16, 32, 64, 128}: the thread-tile kernel
+// above (an item holds 128/d units); every other shape: the one-CTA-per-unit
+// kernel (damp_decode_any.cu).
+cudaError_t launch_decode_step(const PoolDesc& p, const StepArgs& a0, int in_dtype, int gate,
                                cudaStream_t stream) {
-    if (p.d == 128 && codec_of(p.format) != 0 && decode_unit_fits(a, in_dtype, gate)) {
-        StepArgs b = a;
-        b.n_items = a.n * a.H;   // units
-        return launch_decode_unit(b, in_dtype, gate, codec_of(p.format) == 2, stream);
-    }
-    switch (p.d) {
+    StepArgs a = a0;
+    if (p.d_k == 128 && p.d_v == 128 && codec_of(p.format) != 0 &&
+        decode_unit_fits(a, in_dtype, gate))
+        return launch_decode_unit(a, in_dtype, gate, codec_of(p.format) == 2, stream);
+    if (p.d_k != p.d_v || p.d_k > kMaxFastD || (p.d_k & (p.d_k - 1)))
+        return launch_decode_any(a, in_dtype, gate, stream);
+    const int upi = kMaxFastD / p.d_k;
+    a.n_items = (a.n_items + upi - 1) / upi;
+    switch (p.d_k) {
         case 16: return dispatch_fmt<16>(p, a, in_dtype, gate, stream);
         case 32: return dispatch_fmt<32>(p, a, in_dtype, gate, stream);
         case 64: return dispatch_fmt<64>(p, a, in_dtype, gate, stream);

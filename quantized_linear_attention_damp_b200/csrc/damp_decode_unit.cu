@@ -5,28 +5,34 @@
 // kernel in damp_decode.cu ("STEPQuant ...", Appendix Table C2 steps 1, 2,
 // 3, 6 on the DAMP row format); only the work decomposition differs.
 //
-// CTA of 8 warps.  Half-warp k = 2w + hh of warp w owns key rows [8g, 8g + 8)
-// of the unit, g = order[k] from the head's row-group order in the pool header;
-// a lane owns 8 columns, so one row takes 16 lanes.  Each thread keeps its
-// 8 x 8 tile in registers from dequantize to requantize, and the per-row work
-// (directory lookup, scale, k/q values, row maximum, division, stores) is
-// spread over 8 columns.  The two halves of a warp work on different rows, so
-// a format branch runs both paths, each for its half, where the rows differ in
-// format; the order pairs groups whose FP16 rows line up, so that this is
-// rare.  u = k^T S' is summed in the recursive pairwise order: 8 rows per
-// thread as a subtree, then the top four levels over the 16 row groups by
-// group index, whichever half-warp computed them.
+// CTA of 8 warps.  Warp w owns key rows [16w, 16w + 16) of the unit and lane
+// l owns columns [4l, 4l + 4), so every instruction of a warp works on one key
+// row (or one pair of rows): format branches are uniform over the warp, only
+// the bytes a row's format stores are read, and a row maximum is one
+// warp-wide reduction.  Rows 2p and 2p + 1 of the warp share one packed FP32
+// register pair per column (.x = row 2p, .y = row 2p + 1), so the per-row
+// operands of the packed operations (scale, decay, k, q, beta*k, 1/scale)
+// are natural pairs, and the first level of the pairwise sum u = k^T S' is
+// the horizontal add of one packed product.  Each thread keeps its 16 x 4
+// tile in registers from dequantize to requantize.  u is summed in the
+// recursive pairwise order: 16 rows per thread as a subtree (levels 1-4),
+// then the top three levels over the 8 warps.
+//
+// Per-row operands are gathered once per unit into a small table per warp
+// (k, q, beta*k, the row scale, the row's offset in the block, the KDA
+// decay), by half of the warp's lanes, one row each.
 //
 // Two CTAs share an SM whenever three stages fit in half of its shared
-// memory (4 stages at 27 FP16 rows): their barriers are independent, so one CTA's arithmetic fills the
-// other's barrier waits.  While columns are combined, warp 6 writes back the
-// previous unit's block (one bulk store, once the barrier after phase A has
-// ordered every writer's fenced rows before it) and warp 7 refills the
-// pipeline (cp.async.bulk of the block, q, k, v, the KDA decays and the
-// head's row directory into a shared-memory ring of stages completing on
-// mbarriers; no tensor map, no multicast).  A named barrier between the two
-// lets the refill start as soon as the stage's old store has read it.  An
-// item needs two CTA barriers, not three.
+// memory (4 stages at 27 FP16 rows): their barriers are independent, so one
+// CTA's arithmetic fills the other's barrier waits.  While columns are
+// combined, warp 6 writes back the previous unit's block (one bulk store,
+// once the barrier after the first half of the step has ordered every
+// writer's fenced rows before it) and warp 7 refills the pipeline
+// (cp.async.bulk of the block, q, k, v, the KDA decays and the head's row
+// directory into a shared-memory ring of stages completing on mbarriers; no
+// tensor map, no multicast).  A named barrier between the two lets the refill
+// start as soon as the stage's old store has read it.  An item needs two CTA
+// barriers.
 
 #include <cuda_runtime.h>
 
@@ -42,9 +48,10 @@ namespace {
 
 constexpr int kPT = 256;       // threads (8 warps)
 constexpr int kPD = 128;       // d_k = d_v
-constexpr int kPR = 8;         // rows per thread
-constexpr int kPG = 16;        // row groups (half-warps)
-constexpr uint32_t kDirBytes = kDirStride * 4;   // directory + row-group order
+constexpr int kRW = 16;        // key rows per warp
+constexpr int kPP = kRW / 2;   // row pairs per warp
+constexpr int kNW = kPT / 32;  // warps
+constexpr uint32_t kDirBytes = kPD * 4;   // the head's row directory
 
 // Per-unit metadata written by the refill warp into the stage (32 bytes).
 struct PMeta {
@@ -57,6 +64,18 @@ struct PMeta {
 };
 static_assert(sizeof(PMeta) == 32, "PMeta layout");
 
+// Per-warp table of the warp's 16 rows, as pairs (rows 2p, 2p + 1).
+struct RowTab {
+    float4 kq[kPP];      // {k_2p, k_2p+1, q_2p, q_2p+1}
+    float4 bs[kPP];      // {b_2p, b_2p+1, s_2p, s_2p+1}: b = beta*k; s = row scale (1 for FP16 rows)
+    uint2 off[kPP];      // byte offsets of rows 2p, 2p+1 in the block
+    float2 al[kPP];      // KDA decays of rows 2p, 2p+1
+    uint32_t soff[kRW];  // byte offset of each byte row's scale in the block
+    float amax[kRW];     // row maxima of |X| (byte rows)
+    float inv[kRW];      // Q / amax (byte rows; 0 for zero rows)
+};
+static_assert(sizeof(RowTab) % 16 == 0, "RowTab layout");
+
 template <bool BF16>
 __device__ __forceinline__ float in_at(const uint8_t* base, int idx) {
     if constexpr (BF16) {
@@ -67,37 +86,91 @@ __device__ __forceinline__ float in_at(const uint8_t* base, int idx) {
     }
 }
 
-__device__ __forceinline__ float bf16w(const uint32_t* w, int i) {
-    return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+// INT8 code c (byte c of w, two's complement) as the float 2^23 + 128 + code,
+// exactly: wb = w ^ 0x80808080 holds the codes biased to 1..255, and the byte
+// permute places one of them in the low mantissa bits of 2^23.
+__device__ __forceinline__ float i8_biased(uint32_t wb, int c) {
+    return __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7440u | (uint32_t)c));
 }
 
-// 8 byte-row codes (two words) times the row scale: INT8 or FP8 E4M3 codes.
+// The four E4M3 codes of w widened exactly to FP32 (E4M3 is a subset of FP16).
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
+    uint32_t h01, h23;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"((unsigned short)(w & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"((unsigned short)(w >> 16)));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+
+__device__ __forceinline__ void f16x4_to_f32(uint2 h, float (&f)[4]) {
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+
+// Values of one byte row (4 codes) before the scale: INT8 -> 2^23 + 128 + code
+// (the bias is removed by the caller), FP8 -> the E4M3 value.
 template <bool FP8>
-__device__ __forceinline__ void dq_byte8(uint2 w, float s, float2 (&x)[4]) {
+__device__ __forceinline__ void byte_row_raw(uint32_t w, float (&f)[4]) {
     if constexpr (FP8) {
-        dequant_e4m3x4(w.x, s, x[0], x[1]);
-        dequant_e4m3x4(w.y, s, x[2], x[3]);
+        e4m3x4_to_f32(w, f);
     } else {
-        dequant_int8x4_packed(w.x, s, x[0], x[1]);
-        dequant_int8x4_packed(w.y, s, x[2], x[3]);
+        const uint32_t wb = w ^ 0x80808080u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) f[c] = i8_biased(wb, c);
     }
 }
-__device__ __forceinline__ void dq_fp16x8(uint4 h, float2 (&x)[4]) {
-    dequant_fp16x4(make_uint2(h.x, h.y), x[0], x[1]);
-    dequant_fp16x4(make_uint2(h.z, h.w), x[2], x[3]);
+
+// max |v| over 4 values
+__device__ __forceinline__ float absmax4v(float a, float b, float c, float d) {
+    return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
 }
-__device__ __forceinline__ float absmax8(const float2 (&x)[4]) {
-    float m0, m1;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(m0) : "f"(fabsf(x[0].x)), "f"(fabsf(x[0].y)), "f"(fabsf(x[1].x)));
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(m1) : "f"(fabsf(x[1].y)), "f"(fabsf(x[2].x)), "f"(fabsf(x[2].y)));
-    float m;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m0), "f"(m1), "f"(fabsf(x[3].x)));
-    return fmaxf(m, fabsf(x[3].y));
+
+// Codes of one byte row (4 values, row inverse scale inv), packed in a word.
+template <bool FP8>
+__device__ __forceinline__ uint32_t quant_row4(float a, float b, float c, float d, float inv) {
+    if constexpr (FP8) {
+        return quant_e4m3x4(make_float2(a, b), make_float2(c, d), inv);
+    } else {
+        return quant_int8x4(make_float2(a, b), make_float2(c, d), inv);
+    }
+}
+
+// Two byte rows at once (inverse scales as a pair).
+template <bool FP8>
+__device__ __forceinline__ uint2 quant_pair4(const float2 (&x)[4], float2 inv) {
+    if constexpr (FP8) {
+        float2 y[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) y[c] = mul2_rn(x[c], inv);
+        unsigned short e01, e23, o01, o23;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e01) : "f"(y[1].x), "f"(y[0].x));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e23) : "f"(y[3].x), "f"(y[2].x));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(o01) : "f"(y[1].y), "f"(y[0].y));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(o23) : "f"(y[3].y), "f"(y[2].y));
+        // rows stored as zero (inv == 0) have code 0 (not the -0 code 0x80)
+        return make_uint2(inv.x == 0.0f ? 0u : ((uint32_t)e01 | ((uint32_t)e23 << 16)),
+                          inv.y == 0.0f ? 0u : ((uint32_t)o01 | ((uint32_t)o23 << 16)));
+    } else {
+        // RNE of the exact x*inv by one fused multiply-add with 1.5*2^23 (the
+        // low byte of the sum is the two's-complement code; see quant_int8x4)
+        const float2 magic = f2(12582912.0f);
+        float2 y[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) y[c] = __ffma2_rn(x[c], inv, magic);
+        const uint32_t e01 = __byte_perm(__float_as_uint(y[0].x), __float_as_uint(y[1].x), 0x0040);
+        const uint32_t e23 = __byte_perm(__float_as_uint(y[2].x), __float_as_uint(y[3].x), 0x0040);
+        const uint32_t o01 = __byte_perm(__float_as_uint(y[0].y), __float_as_uint(y[1].y), 0x0040);
+        const uint32_t o23 = __byte_perm(__float_as_uint(y[2].y), __float_as_uint(y[3].y), 0x0040);
+        return make_uint2(__byte_perm(e01, e23, 0x5410), __byte_perm(o01, o23, 0x5410));
+    }
 }
 
 template <bool KDA, bool BF16, bool FP8>
 __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     constexpr uint32_t ELT = BF16 ? 2 : 4;
+    constexpr float kQ = FP8 ? 448.0f : 127.0f;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -118,7 +191,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     // U == L (mod 32), loaded 32 units ahead of use.  The ring holds raw
     // values: nothing waits for the loads until the unit is issued, and no
     // branch depends on a freshly loaded slot index.
-    constexpr int kIssueWarp = kPT / 32 - 1;    // refill
+    constexpr int kIssueWarp = kNW - 1;         // refill
     constexpr int kStoreWarp = kIssueWarp - 1;  // write-back
     struct RMeta {
         int slot;          // slot index; INT_MIN: no such unit
@@ -159,6 +232,15 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     RMeta ring{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
     if (warp == kIssueWarp) ring = load_meta(lane);
 
+    // Programmatic dependent launch: everything above touches only this
+    // call's inputs (slot indices, gates, the pool's block table), which no
+    // earlier decode step writes, so it overlaps the previous kernel's tail.
+    // From here on the pool, q/k/v and out are read or written: wait until the
+    // grids this launch depends on have completed and their writes are
+    // visible.  The next launch on the stream may start its own prologue now.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
     // Refill the stage of item il: metadata, then one bulk copy per operand,
     // all completing on the stage's mbarrier (lane 0 issues them).
     auto issue = [&](int il) {
@@ -175,7 +257,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
         r.hb.y = __shfl_sync(0xffffffffu, ring.hb.y, src);
         const PMeta m = finish_meta(r);
         if (lane == src) ring = load_meta(il + 32);
-        if (lane == 0) {
+        if (lane == 0 && !(il == 0 && (a.hooks & kHookHoldFirstItem))) {
             *reinterpret_cast<PMeta*>(st + a.st_meta) = m;
             const uint32_t fb = full_bar(stage);
             if (m.active == 1) {
@@ -187,7 +269,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
                 if constexpr (KDA)
                     bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + (size_t)m.unit * kPD, kPD * 4, fb);
-                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kDirStride, kDirBytes, fb);
+                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kPD, kDirBytes, fb);
             } else {
                 mbar_arrive(fb);
             }
@@ -204,124 +286,157 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     };
 
     const int ahead = NS - 2;
+    int issued = 0;   // items issued so far (meaningful in the refill warp)
     if (warp == kIssueWarp)
-        for (int il = 0; il < ahead && il < my_items; ++il) issue(il);
+        for (; issued < ahead && issued < my_items; ++issued) issue(issued);
 
-    // ---- consumers: half-warp k = 2w + hh of warp w owns row group order[k] of
-    // the unit's head
-    const int hh = lane >> 4;
-    const int cg = lane & 15;           // columns 8cg .. 8cg+7
-
+    // ---- consumers: warp w owns rows [16w, 16w + 16), lane l columns [4l, 4l + 4)
     uint8_t* scratch = smem + a.scratch_off;
-    float* red_u = reinterpret_cast<float*>(scratch);   // [16][128], by row group
-    float* red_w = red_u + kPG * kPD;                   // [16][128], by row group
-    float* delta_s = red_w + kPG * kPD;                 // [128]
-    float* cpart_s = delta_s + kPD;                     // [16], by row group
-    float* rowbuf = cpart_s + kPG + (warp * 2 + hh) * 16;   // this half-warp's 16 floats
+    float* red_u = reinterpret_cast<float*>(scratch);   // [8][128], by warp
+    float* red_w = red_u + kNW * kPD;                   // [8][128], by warp
+    float2* delta2 = reinterpret_cast<float2*>(red_w + kNW * kPD);   // [128] (delta_j, delta_j)
+    float* cpart_s = reinterpret_cast<float*>(delta2 + kPD);        // [8], by warp (16 B padded)
+    RowTab* tab = reinterpret_cast<RowTab*>(cpart_s + 16) + warp;
+    const int row0 = warp * kRW;
 
     int it = 0, stage = 0;
     uint32_t parity = 0;
     bool aborted = false;
     for (; it < my_items; ++it) {
-        const bool ok = mbar_wait_bounded(full_bar(stage), parity);
+        // A warp whose wait gave up in any lane skips the unit; the CTA leaves
+        // the loop together at the first barrier below.
+        const bool ok =
+            __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(stage), parity, a.wait_ns));
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
         const PMeta meta = *reinterpret_cast<const PMeta*>(st + a.st_meta);
-        const bool any = ok && meta.active == 1;
-        // row group of this half-warp (the order is loaded with the directory)
-        const int rg = any ? (st[a.st_dir + kDirWords * 4 + warp * 2 + hh] & (kPG - 1)) : warp * 2 + hh;
-        const int r0 = rg * kPR;            // rows r0 .. r0+7
+        const bool any = ok && meta.active == 1;   // uniform over the warp
         uint8_t* blk = st;
         const uint8_t* sq = st + a.st_q;
         const uint8_t* sk = st + a.st_k;
-        const float* salpha = reinterpret_cast<const float*>(st + a.st_alpha);
-        const uint32_t* sdir = reinterpret_cast<const uint32_t*>(st + a.st_dir) + r0;
-        const uint8_t* b16 = blk + cg * 16;
-        const uint8_t* b8 = blk + cg * 8;
+        const uint32_t* sdir = reinterpret_cast<const uint32_t*>(st + a.st_dir);
+        const uint8_t* b4 = blk + 4 * lane;   // this lane's 4 codes of a byte row
+        const uint8_t* b8 = blk + 8 * lane;   // this lane's 4 values of an FP16 row
 
-        float2 x[kPR][4];
-        uint32_t kw[BF16 ? kPR / 2 : 1], qw[BF16 ? kPR / 2 : 1];
-        auto kval = [&](int i) { return BF16 ? bf16w(kw, i) : in_at<false>(sk, r0 + i); };
-        auto qval = [&](int i) { return BF16 ? bf16w(qw, i) : in_at<false>(sq, r0 + i); };
-        uint32_t dir[kPR];
-        // `any` is uniform over the CTA: the directory (and so every row
-        // offset) is valid only for a loaded unit.
+        float2 x[kPP][4];
+        uint32_t m16 = 0;   // bit i: row row0 + i is an FP16 row
         if (any) {
-            if constexpr (BF16) {
-                const uint4 kv = *reinterpret_cast<const uint4*>(sk + 2 * r0);
-                const uint4 qv = *reinterpret_cast<const uint4*>(sq + 2 * r0);
-                kw[0] = kv.x; kw[1] = kv.y; kw[2] = kv.z; kw[3] = kv.w;
-                qw[0] = qv.x; qw[1] = qv.y; qw[2] = qv.z; qw[3] = qv.w;
-            }
+            // ---- per-row operands of this warp's 16 rows (lanes 0-15, one row each)
             {
-                const uint4 d0 = reinterpret_cast<const uint4*>(sdir)[0];
-                const uint4 d1 = reinterpret_cast<const uint4*>(sdir)[1];
-                dir[0] = d0.x; dir[1] = d0.y; dir[2] = d0.z; dir[3] = d0.w;
-                dir[4] = d1.x; dir[5] = d1.y; dir[6] = d1.z; dir[7] = d1.w;
-            }
-            // ---- step 1: reconstruct S^ (all candidate reads first, then decode)
-#pragma unroll
-            for (int i0 = 0; i0 < kPR; i0 += 4) {
-                uint4 w16[4];
-                uint2 w8[4];
-                float sc[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t e = dir[i0 + j], off = e & 0xffffu;
-                    w16[j] = *reinterpret_cast<const uint4*>(b16 + off);
-                    w8[j] = *reinterpret_cast<const uint2*>(b8 + off);
-                    sc[j] = *reinterpret_cast<const float*>(blk + ((e >> 16) & 0x7fffu));
+                bool f16 = false;
+                float cp = 0.f;
+                if (lane < kRW) {
+                    const int r = row0 + lane;
+                    const uint32_t e = sdir[r];
+                    f16 = (e >> 31) != 0;
+                    const float kr = in_at<BF16>(sk, r), qr = in_at<BF16>(sq, r);
+                    const float br = __fmul_rn(meta.beta, kr);
+                    const uint32_t so = dir_scale(e);
+                    const float sr = f16 ? 1.0f : *reinterpret_cast<const float*>(blk + so);
+                    const int p = lane >> 1, j = lane & 1;
+                    float* kq = reinterpret_cast<float*>(&tab->kq[p]);
+                    float* bs = reinterpret_cast<float*>(&tab->bs[p]);
+                    kq[j] = kr;
+                    kq[2 + j] = qr;
+                    bs[j] = br;
+                    bs[2 + j] = sr;
+                    reinterpret_cast<uint32_t*>(&tab->off[p])[j] = dir_row(e);
+                    if constexpr (KDA)
+                        reinterpret_cast<float*>(&tab->al[p])[j] =
+                            reinterpret_cast<const float*>(st + a.st_alpha)[r];
+                    tab->soff[lane] = so;
+                    cp = __fmul_rn(qr, br);
                 }
+                m16 = __ballot_sync(0xffffffffu, f16);
+                // c = q^T (beta k) over this warp's rows (any order)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (dir[i0 + j] >> 31) dq_fp16x8(w16[j], x[i0 + j]);
-                    else dq_byte8<FP8>(w8[j], sc[j], x[i0 + j]);
-                }
+                for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
+                if (lane == 0) cpart_s[warp] = cp;
+                __syncwarp();
             }
-            // ---- step 2 (first half): S' = D S^; u = k^T S' (pairwise); w = q^T S'
-            float2 stk[3][4];
-            float2 us[4], ws[4];
+            // ---- step 1 (reconstruct) and step 2 (first half), pair by pair:
+            // S' = D S^; u = k^T S' (pairwise); w = q^T S'
+            const float2 al_g = f2(meta.alpha);
+            const float2 bias2 = f2(-8388736.0f);   // -(2^23 + 128)
+            float2 wacc[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) ws[c] = f2(0.f);
+            for (int c = 0; c < 4; ++c) wacc[c] = f2(0.f);
+            float2 stk[3][2];
+            float2 usum[2];
 #pragma unroll
-            for (int i = 0; i < kPR; ++i) {
-                const float al = KDA ? salpha[r0 + i] : meta.alpha;
-                const float kr = kval(i), qr = qval(i);
-                float2 v[4];
+            for (int p = 0; p < kPP; ++p) {
+                const uint32_t fm = (m16 >> (2 * p)) & 3u;   // bit0: row 2p FP16; bit1: row 2p+1
+                const uint2 o = tab->off[p];
+                const float4 bs = tab->bs[p];
+                const float2 sp = make_float2(bs.z, bs.w);
+                if (fm == 0u) {
+                    float e[4], d[4];
+                    byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
+                    byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float2 t = make_float2(e[c], d[c]);
+                        if constexpr (!FP8) t = __fadd2_rn(t, bias2);
+                        x[p][c] = __fmul2_rn(t, sp);
+                    }
+                } else if (fm == 3u) {
+                    float e[4], d[4];
+                    f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.x), e);
+                    f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.y), d);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) x[p][c] = make_float2(e[c], d[c]);
+                } else {
+                    // one FP16 row and one byte row: the FP16 half is offset by
+                    // -0 and scaled by 1 (both exact, signed zeros kept)
+                    float e[4], d[4];
+                    if (fm == 1u) {
+                        f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.x), e);
+                        byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
+                    } else {
+                        byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
+                        f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.y), d);
+                    }
+                    const float2 bz = fm == 1u ? make_float2(-0.0f, -8388736.0f)
+                                               : make_float2(-8388736.0f, -0.0f);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float2 t = make_float2(e[c], d[c]);
+                        if constexpr (!FP8) t = __fadd2_rn(t, bz);
+                        x[p][c] = __fmul2_rn(t, sp);
+                    }
+                }
+                const float2 alp = KDA ? tab->al[p] : al_g;
+                const float4 kq = tab->kq[p];
+                const float2 kp = make_float2(kq.x, kq.y), qp = make_float2(kq.z, kq.w);
+                float L[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    x[i][c] = __fmul2_rn(x[i][c], f2(al));
-                    v[c] = mul2_rn(f2(kr), x[i][c]);      // scalar products: never fused
-                    ws[c] = __ffma2_rn(f2(qr), x[i][c], ws[c]);
+                    x[p][c] = __fmul2_rn(x[p][c], alp);
+                    const float2 pr = __fmul2_rn(kp, x[p][c]);   // fl(k_i S'_ij), two rows
+                    L[c] = __fadd_rn(pr.x, pr.y);                  // level 1 of the pairwise sum
+                    wacc[c] = __ffma2_rn(qp, x[p][c], wacc[c]);
                 }
+                float2 v[2] = {make_float2(L[0], L[1]), make_float2(L[2], L[3])};
 #pragma unroll
-                for (int lv = 0; lv < 3; ++lv) {
-                    if ((i >> lv) & 1) {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) v[c] = __fadd2_rn(stk[lv][c], v[c]);
+                for (int lv = 0; lv < 3; ++lv) {   // levels 2-4 over this warp's pairs
+                    if ((p >> lv) & 1) {
+                        v[0] = __fadd2_rn(stk[lv][0], v[0]);
+                        v[1] = __fadd2_rn(stk[lv][1], v[1]);
                     } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) stk[lv][c] = v[c];
+                        stk[lv][0] = v[0];
+                        stk[lv][1] = v[1];
                         break;
                     }
                 }
-                if (i == kPR - 1) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) us[c] = v[c];
+                if (p == kPP - 1) {
+                    usum[0] = v[0];
+                    usum[1] = v[1];
                 }
             }
-            float* ru = red_u + rg * kPD + 8 * cg;
-            float* rw = red_w + rg * kPD + 8 * cg;
-            reinterpret_cast<float4*>(ru)[0] = make_float4(us[0].x, us[0].y, us[1].x, us[1].y);
-            reinterpret_cast<float4*>(ru)[1] = make_float4(us[2].x, us[2].y, us[3].x, us[3].y);
-            reinterpret_cast<float4*>(rw)[0] = make_float4(ws[0].x, ws[0].y, ws[1].x, ws[1].y);
-            reinterpret_cast<float4*>(rw)[1] = make_float4(ws[2].x, ws[2].y, ws[3].x, ws[3].y);
-            // c = q^T (beta k) over this row group: lane cg < 8 takes row r0 + cg
-            float cp = 0.f;
-            if (cg < kPR) cp = __fmul_rn(in_at<BF16>(sq, r0 + cg),
-                                         __fmul_rn(meta.beta, in_at<BF16>(sk, r0 + cg)));
-#pragma unroll
-            for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
-            if (cg == 0) cpart_s[rg] = cp;
+            reinterpret_cast<float4*>(red_u + warp * kPD)[lane] =
+                make_float4(usum[0].x, usum[0].y, usum[1].x, usum[1].y);
+            reinterpret_cast<float4*>(red_w + warp * kPD)[lane] =
+                make_float4(__fadd_rn(wacc[0].x, wacc[0].y), __fadd_rn(wacc[1].x, wacc[1].y),
+                            __fadd_rn(wacc[2].x, wacc[2].y), __fadd_rn(wacc[3].x, wacc[3].y));
         }
         if (bar_red_or(0, kPT, ok ? 0 : 1)) {
             aborted = true;
@@ -339,99 +454,133 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             if (lane == 0 && it >= 1) store_item(it - 1);
         } else if (warp == kIssueWarp) {
             asm volatile("bar.sync 2, 64;" ::: "memory");
-            if (it + ahead < my_items) issue(it + ahead);
+            if (it + ahead < my_items) {
+                issue(it + ahead);
+                issued = it + ahead + 1;
+            }
         }
         // ---- step 2 (second half) + step 3: delta_j and out_j, 128 columns
+        bool bad = false;   // a non-finite input (checked when a.validate)
         if (tid < kPD) {
             const int j = tid;
             if (meta.active == 1) {
+                if (a.validate) {
+                    const float aj = KDA ? reinterpret_cast<const float*>(st + a.st_alpha)[j] : meta.alpha;
+                    bad = !(isfinite(in_at<BF16>(sq, j)) && isfinite(in_at<BF16>(sk, j)) &&
+                            isfinite(in_at<BF16>(st + a.st_v, j)) && isfinite(aj) &&
+                            isfinite(meta.beta));
+                }
                 const float* c0 = red_u + j;
-                float t[8];
-#pragma unroll
-                for (int q2 = 0; q2 < 8; ++q2)
-                    t[q2] = __fadd_rn(c0[(2 * q2) * kPD], c0[(2 * q2 + 1) * kPD]);
                 const float uj = __fadd_rn(
-                    __fadd_rn(__fadd_rn(t[0], t[1]), __fadd_rn(t[2], t[3])),
-                    __fadd_rn(__fadd_rn(t[4], t[5]), __fadd_rn(t[6], t[7])));
+                    __fadd_rn(__fadd_rn(c0[0 * kPD], c0[1 * kPD]), __fadd_rn(c0[2 * kPD], c0[3 * kPD])),
+                    __fadd_rn(__fadd_rn(c0[4 * kPD], c0[5 * kPD]), __fadd_rn(c0[6 * kPD], c0[7 * kPD])));
                 const float* w0 = red_w + j;
                 float wj = 0.f;
 #pragma unroll
-                for (int q2 = 0; q2 < kPG; ++q2) wj = __fadd_rn(wj, w0[q2 * kPD]);
-                const float4* cpp = reinterpret_cast<const float4*>(cpart_s);
-                float c = 0.f;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 v4 = cpp[q4];
-                    c += (v4.x + v4.y) + (v4.z + v4.w);
-                }
+                for (int q2 = 0; q2 < kNW; ++q2) wj = __fadd_rn(wj, w0[q2 * kPD]);
+                const float4 c4a = reinterpret_cast<const float4*>(cpart_s)[0];
+                const float4 c4b = reinterpret_cast<const float4*>(cpart_s)[1];
+                const float c = ((c4a.x + c4a.y) + (c4a.z + c4a.w)) + ((c4b.x + c4b.y) + (c4b.z + c4b.w));
                 const float vj = in_at<BF16>(st + a.st_v, j);
                 const float dj = __fsub_rn(vj, uj);
-                delta_s[j] = dj;
+                delta2[j] = f2(dj);
                 a.out[(size_t)meta.unit * kPD + j] = __fmaf_rn(c, dj, wj);
             } else if (meta.unit >= 0) {
                 a.out[(size_t)meta.unit * kPD + j] = 0.f;
                 if (j == 0 && meta.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
             }
         }
-        __syncthreads();
+        if (a.validate) {
+            bad = __syncthreads_or(bad);
+            if (bad) {
+                // the unit is skipped: out row zeroed, block neither updated nor stored
+                if (tid < kPD) a.out[(size_t)meta.unit * kPD + tid] = 0.f;
+                if (tid == 0) {
+                    reinterpret_cast<PMeta*>(st + a.st_meta)->active = 0;
+                    atomicOr(a.status, DAMP_EFLAG_NONFINITE);
+                }
+            }
+        } else {
+            __syncthreads();
+        }
 
         // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
-        if (any) {
-            const float4* dp = reinterpret_cast<const float4*>(delta_s + 8 * cg);
-            const float4 d0 = dp[0], d1 = dp[1];
-            const float2 dl[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
-                                  make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
-            float amax[kPR];
-#pragma unroll
-            for (int i = 0; i < kPR; ++i) {
-                const float b = __fmul_rn(meta.beta, kval(i));
-#pragma unroll
-                for (int c = 0; c < 4; ++c) x[i][c] = __ffma2_rn(f2(b), dl[c], x[i][c]);
-                // row maxima of both half-warps with full-warp reductions (the
-                // other half contributes 0, the smallest |x|)
-                const uint32_t mb = __float_as_uint(absmax8(x[i]));
-                const uint32_t m0 = __reduce_max_sync(0xffffffffu, hh ? 0u : mb);
-                const uint32_t m1 = __reduce_max_sync(0xffffffffu, hh ? mb : 0u);
-                amax[i] = __uint_as_float(hh ? m1 : m0);
+        if (any && !bad) {
+            float2 dl[4];
+            {
+                const float4 d0 = reinterpret_cast<const float4*>(delta2 + 4 * lane)[0];
+                const float4 d1 = reinterpret_cast<const float4*>(delta2 + 4 * lane)[1];
+                dl[0] = make_float2(d0.x, d0.y);
+                dl[1] = make_float2(d0.z, d0.w);
+                dl[2] = make_float2(d1.x, d1.y);
+                dl[3] = make_float2(d1.z, d1.w);
             }
-            if (cg == 0) {
-                reinterpret_cast<float4*>(rowbuf)[0] = make_float4(amax[0], amax[1], amax[2], amax[3]);
-                reinterpret_cast<float4*>(rowbuf)[1] = make_float4(amax[4], amax[5], amax[6], amax[7]);
+            float am[kRW];
+#pragma unroll
+            for (int p = 0; p < kPP; ++p) {
+                const uint32_t fm = (m16 >> (2 * p)) & 3u;
+                const float4 bs = tab->bs[p];
+                const float2 bp = make_float2(bs.x, bs.y);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) x[p][c] = __ffma2_rn(bp, dl[c], x[p][c]);
+                am[2 * p] = am[2 * p + 1] = 0.f;
+                if (!(fm & 1u))
+                    am[2 * p] = __uint_as_float(__reduce_max_sync(
+                        0xffffffffu, __float_as_uint(absmax4v(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x))));
+                if (!(fm & 2u))
+                    am[2 * p + 1] = __uint_as_float(__reduce_max_sync(
+                        0xffffffffu, __float_as_uint(absmax4v(x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y))));
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < kRW; i += 4)
+                    *reinterpret_cast<float4*>(&tab->amax[i]) = make_float4(am[i], am[i + 1], am[i + 2], am[i + 3]);
             }
             __syncwarp();
-            if (cg < kPR) {
-                const uint32_t e = sdir[cg];
-                if (!(e >> 31)) {
-                    float scale, inv;
-                    row_scale<FP8>(rowbuf[cg], scale, inv);
-                    rowbuf[kPR + cg] = inv;
-                    *reinterpret_cast<float*>(blk + ((e >> 16) & 0x7fffu)) = scale;
+            // per byte row r = lane & 15: lanes 0-15 form inv = fl(Q/a), lanes
+            // 16-31 scale = fl(a/Q) and store it into the block
+            {
+                const int r = lane & 15;
+                const bool byte_row = !((m16 >> r) & 1u);
+                const float am_r = tab->amax[r];
+                float res = 0.f;
+                if (byte_row) res = lane < 16 ? __fdiv_rn(kQ, am_r) : __fdiv_rn(am_r, kQ);
+                const float inv_r = __shfl_sync(0xffffffffu, res, r);
+                if (byte_row) {
+                    const bool zero = am_r == 0.0f || isinf(inv_r);
+                    if (lane < 16) tab->inv[r] = zero ? 0.0f : res;
+                    else *reinterpret_cast<float*>(blk + tab->soff[r]) = zero ? 0.0f : res;
                 }
             }
             __syncwarp();
-            const float4 i0 = reinterpret_cast<const float4*>(rowbuf)[2];
-            const float4 i1 = reinterpret_cast<const float4*>(rowbuf)[3];
-            const float inv[kPR] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-            {
-                const uint4 d0 = reinterpret_cast<const uint4*>(sdir)[0];
-                const uint4 d1 = reinterpret_cast<const uint4*>(sdir)[1];
-                dir[0] = d0.x; dir[1] = d0.y; dir[2] = d0.z; dir[3] = d0.w;
-                dir[4] = d1.x; dir[5] = d1.y; dir[6] = d1.z; dir[7] = d1.w;
-            }
 #pragma unroll
-            for (int i = 0; i < kPR; ++i) {
-                const uint32_t e = dir[i], off = e & 0xffffu;
-                if (e >> 31) {
-                    const uint2 h0 = quant_fp16x4(x[i][0], x[i][1]);
-                    const uint2 h1 = quant_fp16x4(x[i][2], x[i][3]);
-                    *reinterpret_cast<uint4*>(const_cast<uint8_t*>(b16) + off) =
-                        make_uint4(h0.x, h0.y, h1.x, h1.y);
+            for (int p = 0; p < kPP; ++p) {
+                const uint32_t fm = (m16 >> (2 * p)) & 3u;
+                const uint2 o = tab->off[p];
+                const float2 ip = *reinterpret_cast<const float2*>(&tab->inv[2 * p]);
+                if (fm == 0u) {
+                    const uint2 cw = quant_pair4<FP8>(x[p], ip);
+                    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) = cw.x;
+                    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) = cw.y;
+                } else if (fm == 3u) {
+                    const uint2 he = quant_fp16x4(make_float2(x[p][0].x, x[p][1].x),
+                                                  make_float2(x[p][2].x, x[p][3].x));
+                    const uint2 ho = quant_fp16x4(make_float2(x[p][0].y, x[p][1].y),
+                                                  make_float2(x[p][2].y, x[p][3].y));
+                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.x) = he;
+                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.y) = ho;
+                } else if (fm == 1u) {
+                    const uint2 he = quant_fp16x4(make_float2(x[p][0].x, x[p][1].x),
+                                                  make_float2(x[p][2].x, x[p][3].x));
+                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.x) = he;
+                    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) =
+                        quant_row4<FP8>(x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y, ip.y);
                 } else {
-                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + off) =
-                        FP8 ? make_uint2(quant_e4m3x4(x[i][0], x[i][1], inv[i]),
-                                         quant_e4m3x4(x[i][2], x[i][3], inv[i]))
-                            : make_uint2(quant_int8x4(x[i][0], x[i][1], inv[i]),
-                                         quant_int8x4(x[i][2], x[i][3], inv[i]));
+                    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) =
+                        quant_row4<FP8>(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x, ip.x);
+                    const uint2 ho = quant_fp16x4(make_float2(x[p][0].y, x[p][1].y),
+                                                  make_float2(x[p][2].y, x[p][3].y));
+                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.y) = ho;
                 }
             }
             fence_proxy_async_smem();
@@ -444,18 +593,20 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
 
     // The last completed item (it-1) is still to be written back.
     __syncthreads();
-    if (warp == kStoreWarp && lane == 0) {
-        if (it >= 1) store_item(it - 1);
-        if (aborted) {
-            atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
-            // drain loads that may still be landing in this CTA's stages
-            for (int j = 0; j <= ahead; ++j) {
-                const int jt = it + j;
-                if (jt >= my_items) break;
-                (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
-                                        100000000ull);
+    if (aborted) {
+        // loads still landing in this CTA's stages: the items after the last
+        // one consumed that the refill warp issued (it .. issued-1)
+        if (warp == kIssueWarp) {
+            if (lane == 0) {
+                atomicOr(a.status, DAMP_EFLAG_TIMEOUT);
+                for (int jt = it; jt < issued; ++jt)
+                    (void)mbar_wait_bounded(full_bar(jt % NS), static_cast<uint32_t>(jt / NS) & 1u,
+                                            100000000ull);
             }
         }
+    }
+    if (warp == kStoreWarp && lane == 0) {
+        if (it >= 1) store_item(it - 1);
         bulk_wait_all<0>();
     }
 }
@@ -465,6 +616,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
 uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
     const uint32_t elt = bf16 ? 2 : 4;
     auto up = [](uint32_t x, uint32_t m) { return (x + m - 1) / m * m; };
+    // a block may be read up to 8 bytes per lane past a row: keep 256 bytes of
+    // the stage after the largest block
     uint32_t off = a.block_stride;
     a.st_q = off;
     off = up(off + kPD * elt, 16);
@@ -480,7 +633,8 @@ uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
     a.st_meta = off;
     off += sizeof(PMeta);
     a.stage_bytes = up(off, 128);
-    const uint32_t scratch = up((2 * kPG * kPD + kPD + kPG + kPG * 16) * 4, 128);
+    const uint32_t scratch =
+        up((2 * kNW * kPD + 2 * kPD + 16) * 4 + kNW * (uint32_t)sizeof(RowTab), 128);
     uint32_t ns = (budget - scratch - 128) / a.stage_bytes;
     if (ns > 6) ns = 6;
     if (ns < 3) return 0;
@@ -531,7 +685,20 @@ cudaError_t launch_unit_t(const StepArgs& a0, cudaStream_t stream) {
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int grid = std::min(a.n_items, sms * per_sm);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kPT, smem, stream>>>(a);
+    // launched as a programmatic dependent of the previous kernel on the
+    // stream (the kernel waits for it before touching shared data)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

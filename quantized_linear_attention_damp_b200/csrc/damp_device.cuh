@@ -136,7 +136,7 @@ struct Geo {
 };
 
 // FP16-row bits of rows [r0, r0 + RPT) and the rank of row r0 among FP16 rows.
-// mask = the head's 128-bit FP16-row mask (bit i = key row i is FP16).
+// mask = the first 128 bits of the head's FP16-row mask (bit i = key row i is FP16).
 template <int D>
 __device__ __forceinline__ void row_formats(uint4 mask, int r0, uint32_t& bits, int& rank16) {
     constexpr int RPT = Geo<D>::RPT;
@@ -236,7 +236,9 @@ __device__ __forceinline__ uint32_t quant_e4m3x4(float2 lo, float2 hi, float inv
     unsigned short p01, p23;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(p01) : "f"(a.y), "f"(a.x));
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(p23) : "f"(b.y), "f"(b.x));
-    return (uint32_t)p01 | ((uint32_t)p23 << 16);
+    // a row stored as zero (inv == 0) has code 0 everywhere: x * 0 is -0 for
+    // negative x, whose E4M3 code would be 0x80
+    return inv == 0.0f ? 0u : ((uint32_t)p01 | ((uint32_t)p23 << 16));
 }
 
 // Requantize rows [r0, r0+RPT) of x into a quantized block at `blk` (shared or
@@ -328,12 +330,12 @@ __device__ __forceinline__ void load_tile_gdir(const uint8_t* blk, const uint32_
     for (int i = 0; i < RPT; ++i) e[i] = __ldg(dir + r0 + i);
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-        const uint8_t* row = blk + (e[i] & 0xffffu);
+        const uint8_t* row = blk + dir_row(e[i]);
         if (e[i] >> 31) {
             raw[i] = __ldg(reinterpret_cast<const uint2*>(row + cg * 8));
         } else {
             raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(row + cg * 4));
-            raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(blk + ((e[i] >> 16) & 0x7fffu)));
+            raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(blk + dir_scale(e[i])));
         }
     }
 #pragma unroll
@@ -365,10 +367,10 @@ __device__ __forceinline__ void load_tile_dir(const uint8_t* blk, const uint32_t
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
             e[j] = dir[r0 + i0 + j];
-            const uint8_t* row = blk + (e[j] & 0xffffu);
+            const uint8_t* row = blk + dir_row(e[j]);
             w16[j] = *reinterpret_cast<const uint2*>(row + cg * 8);
             w8[j] = *reinterpret_cast<const uint32_t*>(row + cg * 4);
-            sc[j] = *reinterpret_cast<const float*>(blk + ((e[j] >> 16) & 0x7fffu));
+            sc[j] = *reinterpret_cast<const float*>(blk + dir_scale(e[j]));
         }
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
@@ -398,14 +400,14 @@ __device__ __forceinline__ void store_tile_dir(uint8_t* blk, const uint32_t* dir
             float scale, inv;
             row_scale<FP8>(rowbuf[cg], scale, inv);
             rowbuf[RPT + cg] = inv;
-            *reinterpret_cast<float*>(blk + ((e >> 16) & 0x7fffu)) = scale;
+            *reinterpret_cast<float*>(blk + dir_scale(e)) = scale;
         }
     }
     __syncwarp();
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const uint32_t e = dir[r0 + i];
-        uint8_t* row = blk + (e & 0xffffu);
+        uint8_t* row = blk + dir_row(e);
         if (e >> 31) {
             *reinterpret_cast<uint2*>(row + cg * 8) = quant_fp16x4(x[i][0], x[i][1]);
         } else {

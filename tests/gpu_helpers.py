@@ -42,18 +42,21 @@ class Pair:
     """A GPU pool and an oracle pool built from the same workload."""
 
     def __init__(self, w: W.Workload, fmt: str | None = None, oracle_slots=None,
-                 fp16_map=None):
+                 fp16_map=None, S0=None):
         self.w = w
         self.fmt = fmt or w.fmt
         self.hs = W.head_structure(w.with_(fmt=self.fmt))
         if fp16_map is not None:           # per-head FP16-row counts may differ
             self.is_fp16 = np.ascontiguousarray(fp16_map, np.uint8)
-            self.gpu = D.DampPool("mixed", w.n_slots, w.H, w.d, fp16_map=self.is_fp16)
+            self.gpu = D.DampPool("mixed", w.n_slots, w.H, w.d, fp16_map=self.is_fp16,
+                                  d_v=w.d_v)
         else:
             self.is_fp16 = self.hs.is_fp16
             hp_idx = self.hs.hp_row_idx if self.fmt == "mixed" else None
-            self.gpu = D.DampPool(self.fmt, w.n_slots, w.H, w.d, hp_idx)
-        S0 = W.initial_state(w, range(w.n_slots))
+            self.gpu = D.DampPool(self.fmt, w.n_slots, w.H, w.d, hp_idx, d_v=w.d_v)
+        if S0 is None:
+            S0 = W.initial_state(w, range(w.n_slots))
+        S0 = np.ascontiguousarray(S0, np.float32)
         self.gpu.pack(torch.arange(w.n_slots, dtype=torch.int32, device="cuda"),
                       torch.from_numpy(S0).cuda())
         # oracle: all slots, or only the sampled ones (dict slot -> index)
@@ -66,7 +69,7 @@ class Pair:
     # ---------------------------------------------------------------- steps
     def gpu_step(self, x: W.StepInputs) -> np.ndarray:
         t = torch_inputs(self.w, x)
-        out = torch.empty((self.w.n, self.w.H, self.w.d), dtype=torch.float32, device="cuda")
+        out = torch.empty((self.w.n, self.w.H, self.w.d_v), dtype=torch.float32, device="cuda")
         self.gpu.step(t["slot_idx"], t["q"], t["k"], t["v"], t["alpha"], t["beta"], out)
         torch.cuda.synchronize()
         return out.cpu().numpy()
@@ -126,7 +129,7 @@ class Pair:
         assert dh.max(initial=0) <= 1, "FP16 rows differ by more than 1 ulp"
         assert ds.max(initial=0) <= 1, "scales differ by more than 1 ulp"
         assert dc.max(initial=0) <= 1, "INT8 codes differ by more than 1"
-        n_int8 = int((1 - self.is_fp16).sum()) * self.w.d * len(self.oracle_slots)
+        n_int8 = int((1 - self.is_fp16).sum()) * self.w.d_v * len(self.oracle_slots)
         assert dc.sum() <= max(1, 0.001 * n_int8), "more than 0.1 % of codes differ"
         rep.update(half_diff=int((dh > 0).sum()), scale_diff=int((ds > 0).sum()),
                    code_diff=int((dc > 0).sum()),

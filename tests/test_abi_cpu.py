@@ -79,10 +79,15 @@ def test_layouts_of_other_formats():
 
 def test_pool_bytes():
     n = D.damp_pool_bytes(D.DAMP_FMT_MIXED, 64, 32, 128, 128, 27)
-    # status word; per head a 16-byte FP16-row mask, a 512-byte row directory
-    # followed by its 16-byte row-group order, and a 16-byte block-table entry
-    hdr = 256 * ((16 + 32 * 16 + 32 * (512 + 16) + 32 * 16 + 255) // 256)
+    # status word; per head a 32-byte FP16-row mask, a 4*d_k-byte row
+    # directory and a 16-byte block-table entry; rounded up to 256 bytes
+    hdr = 256 * ((16 + 32 * 32 + 32 * 512 + 32 * 16 + 255) // 256)
     assert n == hdr + 64 * 32 * 20256
+    n = D.damp_pool_bytes(D.DAMP_FMT_MIXED, 3, 5, 256, 48, 9)
+    hdr = 256 * ((16 + 5 * 32 + 5 * 1024 + 5 * 16 + 255) // 256)
+    r = 256 - 9
+    stride = 16 * ((16 * ((4 * r + 15) // 16) + 2 * 9 * 48 + r * 48 + 15) // 16)
+    assert n == hdr + 3 * 5 * stride
 
 
 @pytest.mark.parametrize("args,status", [
@@ -92,14 +97,31 @@ def test_pool_bytes():
     ((D.DAMP_FMT_MIXED, 128, 128, -1), D.DAMP_ERR_INVALID_ARGUMENT),
     ((D.DAMP_FMT_INT8_ROW, 128, 128, 3), D.DAMP_ERR_INVALID_ARGUMENT),
     ((D.DAMP_FMT_FP32, 128, 128, 1), D.DAMP_ERR_INVALID_ARGUMENT),
-    ((D.DAMP_FMT_MIXED, 128, 64, 0), D.DAMP_ERR_UNSUPPORTED),
-    ((D.DAMP_FMT_MIXED, 48, 48, 0), D.DAMP_ERR_UNSUPPORTED),
-    ((D.DAMP_FMT_MIXED, 256, 256, 0), D.DAMP_ERR_UNSUPPORTED),
+    ((D.DAMP_FMT_MIXED, 128, 120, 0), D.DAMP_ERR_UNSUPPORTED),    # d_v not a multiple of 16
+    ((D.DAMP_FMT_MIXED, 8, 8, 0), D.DAMP_ERR_UNSUPPORTED),
+    ((D.DAMP_FMT_MIXED, 272, 272, 0), D.DAMP_ERR_UNSUPPORTED),
+    ((D.DAMP_FMT_FP32, 128, 264, 0), D.DAMP_ERR_UNSUPPORTED),
+    ((D.DAMP_FMT_INT8_ROW, 0, 128, 0), D.DAMP_ERR_UNSUPPORTED),
 ])
 def test_layout_rejects_bad_shapes(args, status):
     with pytest.raises(D.DampError) as ei:
         D.damp_layout(*args)
     assert ei.value.status == status
+
+
+def test_layout_accepts_every_supported_shape():
+    """d_k, d_v in {16, 32, ..., 256}, square or not: block sizes from the
+    format's definition (FP32: 4 d_k d_v; quantized: 4r + 2 hp d_v + r d_v
+    with r = d_k - hp), strides padded to 16 bytes."""
+    for d_k in range(16, 257, 16):
+        for d_v in range(16, 257, 16):
+            assert D.damp_layout(D.DAMP_FMT_FP32, d_k, d_v, 0)[0] == 4 * d_k * d_v
+            for hp in (0, d_k // 3, d_k):
+                b, s = D.damp_layout(D.DAMP_FMT_MIXED, d_k, d_v, hp)
+                r = d_k - hp
+                assert b == 4 * r + 2 * hp * d_v + r * d_v
+                assert s % 16 == 0 and b <= s < b + 32
+            assert D.damp_layout(D.DAMP_FMT_FP8_ROW, d_k, d_v, 0)[0] == 4 * d_k + d_k * d_v
 
 
 def test_status_strings():
@@ -147,23 +169,24 @@ def test_host_only_descriptor_rejects_device_calls():
         D.damp_pool_destroy(h)
 
 
-@pytest.mark.parametrize("d,hp", [(16, 4), (64, 0), (128, 27), (128, 128)])
-def test_block_logical_round_trip(d, hp):
-    g = np.random.default_rng(d + hp)
+@pytest.mark.parametrize("d,dv,hp", [(16, 16, 4), (64, 64, 0), (128, 128, 27), (128, 128, 128),
+                                     (48, 80, 7), (256, 32, 100), (32, 256, 32)])
+def test_block_logical_round_trip(d, dv, hp):
+    g = np.random.default_rng(d + dv + hp)
     H = 3
     idx = np.stack([np.sort(g.permutation(d)[:hp]) for _ in range(H)])
-    h = D.damp_pool_create(D.DAMP_FMT_MIXED, 2, H, d, d, hp, idx if hp else None, None)
+    h = D.damp_pool_create(D.DAMP_FMT_MIXED, 2, H, d, dv, hp, idx if hp else None, None)
     try:
-        _, stride = D.damp_layout(D.DAMP_FMT_MIXED, d, d, hp)
+        _, stride = D.damp_layout(D.DAMP_FMT_MIXED, d, dv, hp)
         for head in range(H):
             is16 = np.zeros(d, bool)
             is16[idx[head]] = True
             scale = np.where(is16, 0, g.uniform(0.1, 2, d)).astype(np.float32)
-            half = np.where(is16[:, None], g.integers(0, 0x7C00, (d, d)), 0).astype(np.uint16)
-            code = np.where(is16[:, None], 0, g.integers(-127, 128, (d, d))).astype(np.int8)
+            half = np.where(is16[:, None], g.integers(0, 0x7C00, (d, dv)), 0).astype(np.uint16)
+            code = np.where(is16[:, None], 0, g.integers(-127, 128, (d, dv))).astype(np.int8)
             raw = D.damp_block_from_logical(h, head, stride, scale=scale, half=half, code=code)
             assert raw.size == stride
-            back = D.damp_block_to_logical(h, head, raw, D.DAMP_FMT_MIXED, d)
+            back = D.damp_block_to_logical(h, head, raw, D.DAMP_FMT_MIXED, d, dv)
             assert np.array_equal(back["scale"], scale)
             assert np.array_equal(back["half"], half)
             assert np.array_equal(back["code"], code)
@@ -171,9 +194,9 @@ def test_block_logical_round_trip(d, hp):
             r = d - hp
             assert np.array_equal(raw[:4 * r].view(np.float32), scale[~is16])
             f16_off = (4 * r + 15) // 16 * 16
-            assert np.array_equal(raw[f16_off:f16_off + 2 * hp * d].view(np.uint16),
+            assert np.array_equal(raw[f16_off:f16_off + 2 * hp * dv].view(np.uint16),
                                   half[is16].reshape(-1))
-            assert np.array_equal(raw[f16_off + 2 * hp * d:f16_off + 2 * hp * d + r * d]
+            assert np.array_equal(raw[f16_off + 2 * hp * dv:f16_off + 2 * hp * dv + r * dv]
                                   .view(np.int8), code[~is16].reshape(-1))
     finally:
         D.damp_pool_destroy(h)
@@ -231,64 +254,60 @@ def test_validate_slots():
         assert ei.value.status == D.DAMP_ERR_INVALID_ARGUMENT and f"entry {pos}" in str(ei.value)
 
 
-def _group_masks(is16_row):
-    return [int(sum(int(is16_row[8 * g + i]) << i for i in range(8))) for g in range(16)]
+# ---------------------------------------------------------------- binding checks
+
+def _host_pool(fmt=D.DAMP_FMT_MIXED, n_slots=4, H=2, d=16, hp=4):
+    """A host-only descriptor (no device buffer): enough for the binding's
+    argument checks, which all run before anything would be enqueued."""
+    idx = np.tile(np.arange(hp, dtype=np.uint16), (H, 1)) if hp else None
+    return D.damp_pool_create(fmt, n_slots, H, d, d, hp, idx, None)
 
 
-def _pair_cost(m, order):
-    return sum(bin(m[order[2 * k]] ^ m[order[2 * k + 1]]).count("1") for k in range(8))
+def _step_tensors(n=3, H=2, d=16, kda=False, dtype=None):
+    import torch
+    dtype = dtype or torch.float32
+    return dict(slot_idx=torch.arange(n, dtype=torch.int32),
+                q=torch.zeros((n, H, d), dtype=dtype), k=torch.zeros((n, H, d), dtype=dtype),
+                v=torch.zeros((n, H, d), dtype=dtype),
+                alpha=torch.zeros((n, H, d) if kda else (n, H)), beta=torch.zeros((n, H)),
+                out=torch.zeros((n, H, d)))
 
 
-def _min_pair_cost(m):
-    """Minimum over all perfect matchings of the 16 groups, by recursion over
-    the lowest unmatched group (memoised on the set of matched groups)."""
-    import functools
-
-    @functools.lru_cache(None)
-    def f(left):
-        if not left:
-            return 0
-        i, rest = left[0], left[1:]
-        return min(bin(m[i] ^ m[j]).count("1") + f(rest[:t] + rest[t + 1:])
-                   for t, j in enumerate(rest))
-    return f(tuple(range(16)))
-
-
-def test_row_group_order_is_a_minimum_cost_pairing():
-    """The d = 128 decode step's row-group order: a permutation of the 16
-    groups whose warp pairs differ in format at the fewest row positions."""
-    g = np.random.default_rng(7)
-    H, d = 6, 128
-    m = np.zeros((H, d), np.uint8)
-    for head, c in enumerate([0, 1, 27, 40, 64, 128]):
-        m[head, g.choice(d, c, replace=False)] = 1
-    h = D.damp_pool_create_map(3, H, d, d, m, None)
+@pytest.mark.parametrize("bad", ["q", "k", "v", "beta", "out", "alpha"])
+def test_binding_rejects_wrong_shapes_before_launch(bad):
+    """The C ABI cannot see tensor sizes: the binding checks every tensor of a
+    step against (n, H, d_k, d_v) of the pool and raises before any call."""
+    import torch
+    h = _host_pool()
     try:
-        for head in range(H):
-            order = D.damp_pool_row_groups(h, head)
-            assert sorted(order) == list(range(16))
-            gm = _group_masks(m[head])
-            assert _pair_cost(gm, order) == _min_pair_cost(gm)
-            lows = [min(order[2 * k], order[2 * k + 1]) for k in range(8)]
-            assert lows == sorted(lows) and all(order[2 * k] < order[2 * k + 1] for k in range(8))
-        # no FP16 row, or every row FP16: nothing to pair, groups in order
-        assert D.damp_pool_row_groups(h, 0) == list(range(16))
-        assert D.damp_pool_row_groups(h, 5) == list(range(16))
-        with pytest.raises(D.DampError):
-            D.damp_pool_row_groups(h, H)
+        t = _step_tensors()
+        t[bad] = torch.zeros((3, 2, 15)) if bad != "beta" else torch.zeros((3, 3))
+        with pytest.raises(ValueError, match=bad):
+            D.damp_decode_step(h, **t)
+        t = _step_tensors()
+        t["slot_idx"] = torch.arange(4, dtype=torch.int32)        # n = 4 vs tensors of 3
+        with pytest.raises(ValueError):
+            D.damp_decode_step(h, **t)
     finally:
         D.damp_pool_destroy(h)
 
 
-def test_row_group_order_worked_example():
-    """Groups 0 and 2 hold FP16 rows at the same 8 positions, all others none:
-    0 pairs with 2 at no cost, then 1 with its lowest free partner 3, and the
-    rest in order."""
-    row = np.zeros(128, np.uint8)
-    row[0:8] = 1
-    row[16:24] = 1
-    h = D.damp_pool_create_map(1, 1, 128, 128, row[None, :], None)
+def test_binding_gate_from_alpha_shape_and_device_checks():
+    import torch
+    h = _host_pool()
     try:
-        assert D.damp_pool_row_groups(h, 0) == [0, 2, 1, 3] + list(range(4, 16))
+        # correct shapes (GDN and KDA) pass the shape checks and stop at the
+        # device check: these tensors are on the CPU
+        for kda in (False, True):
+            with pytest.raises(ValueError, match="CUDA"):
+                D.damp_decode_step(h, **_step_tensors(kda=kda))
+        t = _step_tensors()
+        t["alpha"] = torch.zeros((3, 2, 1))
+        with pytest.raises(ValueError, match="alpha"):
+            D.damp_decode_step(h, **t)
+        with pytest.raises(ValueError, match="state"):
+            D.damp_pool_pack(h, torch.arange(3, dtype=torch.int32), torch.zeros((3, 2, 16, 8)))
+        with pytest.raises(ValueError, match="unknown pool"):
+            D.damp_decode_step(12345, **_step_tensors())
     finally:
         D.damp_pool_destroy(h)

@@ -268,3 +268,54 @@ def test_argument_errors_enqueue_nothing():
         assert torch.equal(before, p.gpu.blocks())
     finally:
         p.close()
+
+
+# ---------------------------------------------------------------- every shape
+
+SHAPES = [(48, 48), (96, 96), (256, 256), (64, 128), (128, 64), (48, 80), (256, 32), (32, 256),
+          (112, 144)]
+
+
+@pytest.mark.parametrize("dk,dv", SHAPES)
+@pytest.mark.parametrize("fmt", ["mixed", "int8", "fp8", "fp32"])
+def test_every_shape_all_formats(dk, dv, fmt):
+    """d_k x d_v states outside the square fast shapes (one CTA per unit):
+    whole state bit-exact and readout within tolerance at every step, GDN and
+    KDA, bf16 and fp32 inputs, a ragged batch (not every slot stepped)."""
+    i = SHAPES.index((dk, dv))
+    w = W.Workload(f"shape_{dk}x{dv}", n=5, n_slots=6, H=3, d=dk, dv=dv, hp=max(1, dk // 5),
+                   steps=3, gate=W.GATE_KDA if i % 2 else W.GATE_GDN,
+                   in_dtype="f32" if i % 3 == 2 else "bf16")
+    run_full(w, fmt, 3)
+
+
+@pytest.mark.parametrize("dk,dv", [(48, 80), (256, 256)])
+def test_every_shape_per_head_fp16_row_counts(dk, dv):
+    w = W.Workload(f"shape_map_{dk}x{dv}", n=4, n_slots=5, H=5, d=dk, dv=dv, hp=0, steps=2,
+                   gate=W.GATE_GDN, in_dtype="bf16")
+    counts = [0, dk, dk // 3, 1, dk - 1]
+    run_full(w, "mixed", 2, fp16_map=random_map(w.H, dk, counts, dk + dv))
+
+
+def test_every_shape_unpack_and_read_raw():
+    """Unpack of a non-square pool equals the oracle's reconstruction, and
+    damp_pool_read_raw returns each block's logical form."""
+    w = W.Workload("shape_unpack", n=4, n_slots=4, H=2, d=96, dv=160, hp=20, steps=1,
+                   gate=W.GATE_GDN, in_dtype="bf16")
+    p = Pair(w, "mixed")
+    try:
+        x = W.step_inputs(w, 0, p.hs)
+        p.gpu_step(x)
+        p.oracle_step_full(x)
+        out = torch.empty((w.n_slots, w.H, w.d, w.d_v), dtype=torch.float32, device="cuda")
+        p.gpu.unpack(torch.arange(w.n_slots, dtype=torch.int32, device="cuda"), out)
+        ref = O.unpack(p.ora, p.is_fp16[None])
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+        for s in range(w.n_slots):
+            for h in range(w.H):
+                lg = D.damp_pool_read_raw(p.gpu.handle, s, h)
+                assert np.array_equal(lg["code"], p.ora.code[s, h])
+                assert np.array_equal(lg["half"], p.ora.half[s, h])
+                assert np.array_equal(lg["scale"].view(np.uint32), p.ora.scale[s, h].view(np.uint32))
+    finally:
+        p.close()

@@ -90,3 +90,103 @@ def test_checkpoint_and_resume():
     assert ds.max() <= 1
     for p in (a, b, c):
         p.close()
+
+
+# ---------------------------------------------------------------- failure paths
+
+def _small(d, gate=W.GATE_GDN, in_dtype=None):
+    return W.Workload(f"fail_d{d}_{gate}", n=6, n_slots=8, H=3, d=d, hp=d // 5, steps=2,
+                      gate=gate, in_dtype=in_dtype or ("f32" if d == 16 else "bf16"))
+
+
+@pytest.mark.parametrize("d,fmt", [(16, "mixed"), (128, "mixed"), (128, "fp8"), (128, "fp32")])
+def test_bounded_wait_runs_out_and_the_kernel_returns(d, fmt):
+    """A pipeline wait that runs out, made on purpose: with
+    DAMP_HOOK_HOLD_FIRST_ITEM every CTA leaves its first item unloaded, and the
+    wait for it is bounded at 5 ms.  The kernel sets DAMP_EFLAG_TIMEOUT, waits
+    (bounded) for its other copies in flight and returns: the stream drains,
+    no block is written, and the next normal steps on the same pool match the
+    oracle bit for bit (the context stays usable)."""
+    import time
+
+    from tests.gpu_helpers import Pair
+    w = _small(d)
+    p = Pair(w, fmt)
+    try:
+        x = W.step_inputs(w, 0, p.hs)
+        before = p.gpu.slots().clone()
+        D.damp_set_test_hooks(5_000_000, D.DAMP_HOOK_HOLD_FIRST_ITEM)
+        try:
+            t0 = time.time()
+            p.gpu_step(x)                      # synchronises
+            elapsed = time.time() - t0
+        finally:
+            D.damp_set_test_hooks(0, 0)
+        assert elapsed < 5.0
+        assert p.gpu.get_error(clear=True) == D.DAMP_EFLAG_TIMEOUT
+        assert p.gpu.get_error() == 0
+        assert torch.equal(before, p.gpu.slots())
+        for s in range(2):
+            x = W.step_inputs(w, s, p.hs)
+            p.check_out(p.gpu_step(x), p.oracle_step_full(x))
+            assert p.check_state()["exact"], s
+        assert p.gpu.get_error() == 0
+    finally:
+        p.close()
+
+
+def _plant(x, name, b, h, j, value):
+    """Set one input element (its float value and, for bf16 inputs, its bits)."""
+    arr = getattr(x, name)
+    if name in ("alpha", "beta"):
+        arr[(b, h) if arr.ndim == 2 else (b, h, j)] = value
+        return
+    arr[b, h, j] = value
+    bits = getattr(x, name + "_bits")
+    if bits is not None:
+        bits[b, h, j] = np.float32(value).view(np.uint32) >> 16
+
+
+@pytest.mark.parametrize("d,fmt,gate", [(16, "mixed", W.GATE_GDN), (16, "int8", W.GATE_KDA),
+                                        (128, "mixed", W.GATE_GDN), (128, "mixed", W.GATE_KDA),
+                                        (128, "fp8", W.GATE_GDN), (128, "fp32", W.GATE_KDA)])
+def test_nonfinite_inputs_are_skipped_and_flagged(d, fmt, gate):
+    """damp_decode_step_validated: units whose q, k, v, alpha or beta hold a
+    NaN or an infinity are skipped (out row zero, block untouched) and flagged
+    with DAMP_EFLAG_NONFINITE; every other unit is stepped exactly as the
+    oracle steps it.  The plain step on clean inputs sets no flag."""
+    from tests.gpu_helpers import Pair
+    w = _small(d, gate)
+    p = Pair(w, fmt)
+    try:
+        x = W.step_inputs(w, 0, p.hs)
+        bad = {(1, 0): ("q", 3, np.nan), (2, 1): ("v", d - 1, np.inf), (0, 2): ("beta", 0, np.nan),
+               (3, 0): ("alpha", 5, np.inf), (4, 1): ("k", 0, -np.inf)}
+        for (b, h), (name, j, val) in bad.items():
+            _plant(x, name, b, h, j, val)
+        t = torch_inputs(w, x)
+        out = torch.full((w.n, w.H, w.d), 3.0, dtype=torch.float32, device="cuda")
+        p.gpu.step(t["slot_idx"], t["q"], t["k"], t["v"], t["alpha"], t["beta"], out,
+                   check_inputs=True)
+        out_g = out.cpu().numpy()
+        # the oracle steps the clean units only
+        res = {}
+        gate_o = 1 if gate == W.GATE_KDA else 0
+        for b, slot in enumerate(x.slot_idx):
+            for h in range(w.H):
+                if (b, h) in bad:
+                    assert not out_g[b, h].any()
+                    continue
+                st = p.ora[int(slot), h]
+                import oracle as O
+                res[(b, h)] = O.step_unit(st, gate_o, p.is_fp16[h], x.q[b, h], x.k[b, h],
+                                          x.v[b, h], x.alpha[b, h], x.beta[b, h])
+        p.check_out(out_g, res)
+        assert p.check_state()["exact"]
+        assert p.gpu.get_error(clear=True) == D.DAMP_EFLAG_NONFINITE
+        x2 = W.step_inputs(w, 1, p.hs)
+        p.check_out(p.gpu_step(x2), p.oracle_step_full(x2))
+        assert p.check_state()["exact"]
+        assert p.gpu.get_error() == 0
+    finally:
+        p.close()

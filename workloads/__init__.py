@@ -50,7 +50,7 @@ class Workload:
     n: int            # batch entries per step
     n_slots: int      # slots in the pool
     H: int
-    d: int            # d_k = d_v
+    d: int            # d_k (and d_v, unless dv is set)
     hp: int           # FP16 rows per head (0 = uniform INT8)
     steps: int
     gate: str         # "gdn" | "kda"
@@ -58,10 +58,15 @@ class Workload:
     fmt: str = "mixed"  # "mixed" | "int8" | "fp8" | "fp32"
     tiny: bool = False
     seed: int = 0
+    dv: int = 0         # d_v when it differs from d (= d_k); 0: d_v = d
 
     @property
     def units(self) -> int:
         return self.n * self.H
+
+    @property
+    def d_v(self) -> int:
+        return self.dv or self.d
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -119,7 +124,7 @@ def head_structure(w: Workload) -> HeadStructure:
     g = rng(w, "heads")
     if w.tiny:
         row_mult = np.ones((H, d))
-        col_mult = np.ones((H, d))
+        col_mult = np.ones((H, w.d_v))
         for h in range(H):
             rows = g.permutation(d)[:2]
             row_mult[h, rows] = 10.0
@@ -127,9 +132,9 @@ def head_structure(w: Workload) -> HeadStructure:
         decay_a = np.zeros(H)
     else:
         row_mult = g.lognormal(0.0, 1.0, size=(H, d))
-        col_mult = np.ones((H, d))
+        col_mult = np.ones((H, w.d_v))
         for h in range(H):
-            col_mult[h, g.permutation(d)[:4]] = 8.0
+            col_mult[h, g.permutation(w.d_v)[:4]] = 8.0
         tiny_alpha = None
         shape = (H, d) if w.gate == GATE_KDA else (H,)
         half_life = np.exp(g.uniform(np.log(1.0), np.log(4096.0), size=shape))
@@ -158,15 +163,15 @@ def head_structure(w: Workload) -> HeadStructure:
 
 
 def initial_state(w: Workload, slots, _structure=None) -> np.ndarray:
-    """FP32 initial states [len(slots)][H][d][d] of the given pool slots."""
+    """FP32 initial states [len(slots)][H][d][d_v] of the given pool slots."""
     if _structure is None:
         hs = head_structure(w)
         row_mult, col_mult = hs.row_mult, hs.col_mult
     else:
         row_mult, col_mult = _structure
-    out = np.empty((len(slots), w.H, w.d, w.d), np.float32)
+    out = np.empty((len(slots), w.H, w.d, w.d_v), np.float32)
     for i, s in enumerate(slots):
-        z = rng(w, "state", int(s)).standard_normal((w.H, w.d, w.d))
+        z = rng(w, "state", int(s)).standard_normal((w.H, w.d, w.d_v))
         out[i] = (0.1 * z * row_mult[:, :, None] * col_mult[:, None, :]).astype(np.float32)
     return out
 
@@ -194,7 +199,7 @@ def step_inputs(w: Workload, step: int, hs: HeadStructure | None = None) -> Step
         slot_idx = g.permutation(w.n_slots)[:n].astype(np.int32)
     q = g.standard_normal((n, H, d))
     k = g.standard_normal((n, H, d))
-    v = g.standard_normal((n, H, d))
+    v = g.standard_normal((n, H, w.d_v))
     q = (q / np.linalg.norm(q, axis=-1, keepdims=True)).astype(np.float32)
     k = (k / np.linalg.norm(k, axis=-1, keepdims=True)).astype(np.float32)
     v = v.astype(np.float32)
