@@ -54,12 +54,28 @@ def _rank_main(rank, port, result_q):
             outs.append(torch.from_numpy(full))
         out = torch.stack(outs)
         dist.all_reduce(out)          # disjoint shards: the sum is the concatenation
+        # the rank's shard in libdamp's own block layout (host-only descriptor):
+        # raw slot bytes encoded from the rank's logical state, gathered by slot
+        import quantized_linear_attention_damp_b200 as D
+        hd = D.damp_pool_create(D.DAMP_FMT_MIXED, len(mine), w.H, w.d, w.d, w.hp, hs.hp_row_idx,
+                                None)
+        try:
+            _, stride = D.damp_layout(D.DAMP_FMT_MIXED, w.d, w.d, w.hp)
+            raw = torch.zeros((w.n_slots, w.H, stride), dtype=torch.int32)
+            for i, slot in enumerate(mine):
+                for h in range(w.H):
+                    blk = D.damp_block_from_logical(hd, h, stride, scale=pool.scale[i, h],
+                                                    half=pool.half[i, h], code=pool.code[i, h])
+                    raw[slot, h] = torch.from_numpy(blk.astype(np.int32))
+        finally:
+            D.damp_pool_destroy(hd)
+        dist.all_reduce(raw)
         state = torch.zeros((w.n_slots, w.H, w.d, w.d), dtype=torch.int32)
         state[mine] = torch.from_numpy(pool.code.astype(np.int32))
         dist.all_reduce(state)
         t = bench.max_over_ranks(0.5 + rank, WORLD)
         if rank == 0:
-            result_q.put((out.numpy(), state.numpy(), t))
+            result_q.put((out.numpy(), state.numpy(), t, raw.numpy()))
     finally:
         dist.destroy_process_group()
 
@@ -71,7 +87,7 @@ def test_two_gloo_ranks_match_unsharded_oracle():
     procs = [ctx.Process(target=_rank_main, args=(r, port, q)) for r in range(WORLD)]
     for p in procs:
         p.start()
-    out, codes, t = q.get(timeout=240)
+    out, codes, t, raw = q.get(timeout=240)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -87,6 +103,18 @@ def test_two_gloo_ranks_match_unsharded_oracle():
         assert np.array_equal(out[s], o)
     assert np.array_equal(codes, pool.code.astype(np.int32))
     assert t == pytest.approx(1.5)
+    # the gathered raw shards are the unsharded pool's blocks, byte for byte
+    import quantized_linear_attention_damp_b200 as D
+    hd = D.damp_pool_create(D.DAMP_FMT_MIXED, w.n_slots, w.H, w.d, w.d, w.hp, hs.hp_row_idx, None)
+    try:
+        _, stride = D.damp_layout(D.DAMP_FMT_MIXED, w.d, w.d, w.hp)
+        for slot in range(w.n_slots):
+            for h in range(w.H):
+                blk = D.damp_block_from_logical(hd, h, stride, scale=pool.scale[slot, h],
+                                                half=pool.half[slot, h], code=pool.code[slot, h])
+                assert np.array_equal(raw[slot, h].astype(np.uint8), blk)
+    finally:
+        D.damp_pool_destroy(hd)
 
 
 def test_rank_workloads_differ_only_in_seed():

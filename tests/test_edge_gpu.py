@@ -75,8 +75,11 @@ def edge_case(d, fmt, gate, in_dtype, overflow, seed=0):
         # head 1: zero row, row too small for 127/a, subnormal-scale row, FP16 subnormals
         S0[s, 1, ZERO] = 0.0
         S0[s, 1, TINY] = g.standard_normal(d) * 1e-38
-        sub = g.standard_normal(d) * 3e-37
-        sub[0] = 1e-36
+        # absmax where the scale a/Q is an FP32 subnormal and Q/a is finite:
+        # Q = 127 needs a in (3.7e-37, 1.5e-36), Q = 448 (FP8) a in (1.3e-36, 5.3e-36)
+        amax_sub = 3e-36 if fmt == "fp8" else 1e-36
+        sub = g.standard_normal(d) * 0.3 * amax_sub
+        sub[0] = amax_sub
         sub[1:4] = [1e-40, -3e-41, 7e-45]
         S0[s, 1, SUB] = sub
         S0[s, 1, F16SUB] = g.standard_normal(d) * 3e-6

@@ -319,3 +319,49 @@ def test_every_shape_unpack_and_read_raw():
                 assert np.array_equal(lg["scale"].view(np.uint32), p.ora.scale[s, h].view(np.uint32))
     finally:
         p.close()
+
+
+@pytest.mark.parametrize("gate", [W.GATE_GDN, W.GATE_KDA])
+def test_sharded_pools_match_one_pool(gate):
+    """The data-parallel split a multi-GPU run uses, on one GPU: two pools
+    holding alternate slots of a workload, each stepped with its own entries
+    of the batch, give bit for bit the out rows and the states of one pool
+    holding every slot (units are independent; no exchange is needed)."""
+    w = W.Workload(f"shard_{gate}", n=8, n_slots=8, H=4, d=128, hp=27, steps=3, gate=gate,
+                   in_dtype="bf16")
+    hs = W.head_structure(w)
+    S0 = torch.from_numpy(W.initial_state(w, range(w.n_slots))).cuda()
+    whole = D.DampPool("mixed", w.n_slots, w.H, w.d, hs.hp_row_idx)
+    whole.pack(torch.arange(w.n_slots, dtype=torch.int32, device="cuda"), S0)
+    owned = [list(range(r, w.n_slots, 2)) for r in range(2)]
+    shards = []
+    for mine in owned:
+        p = D.DampPool("mixed", len(mine), w.H, w.d, hs.hp_row_idx)
+        p.pack(torch.arange(len(mine), dtype=torch.int32, device="cuda"),
+               S0[torch.tensor(mine, device="cuda")].contiguous())
+        shards.append(p)
+    try:
+        for s in range(w.steps):
+            x = W.step_inputs(w, s, hs)
+            t = torch_inputs(w, x)
+            out = torch.empty((w.n, w.H, w.d), dtype=torch.float32, device="cuda")
+            whole.step(t["slot_idx"], t["q"], t["k"], t["v"], t["alpha"], t["beta"], out)
+            out_sh = torch.full_like(out, float("nan"))
+            for mine, p in zip(owned, shards):
+                sel = [b for b in range(w.n) if int(x.slot_idx[b]) in mine]
+                ib = torch.tensor(sel, device="cuda")
+                local = torch.tensor([mine.index(int(x.slot_idx[b])) for b in sel],
+                                     dtype=torch.int32, device="cuda")
+                o = torch.empty((len(sel), w.H, w.d), dtype=torch.float32, device="cuda")
+                p.step(local, t["q"][ib].contiguous(), t["k"][ib].contiguous(),
+                       t["v"][ib].contiguous(), t["alpha"][ib].contiguous(),
+                       t["beta"][ib].contiguous(), o)
+                out_sh[ib] = o
+            torch.cuda.synchronize()
+            assert torch.equal(out, out_sh), s
+        for mine, p in zip(owned, shards):
+            assert torch.equal(whole.slots()[torch.tensor(mine, device="cuda")], p.slots())
+    finally:
+        whole.close()
+        for p in shards:
+            p.close()
