@@ -359,8 +359,12 @@ def test_sharded_pools_match_one_pool(gate):
                 out_sh[ib] = o
             torch.cuda.synchronize()
             assert torch.equal(out, out_sh), s
+        # the states, compared in their logical form (a block's 16-byte padding
+        # is never written and holds whatever each buffer held)
         for mine, p in zip(owned, shards):
-            assert torch.equal(whole.slots()[torch.tensor(mine, device="cuda")], p.slots())
+            lw, ls = whole.read_logical(mine), p.read_logical()
+            for f in ("scale", "half", "code"):
+                assert np.array_equal(lw[f], ls[f]), f
     finally:
         whole.close()
         for p in shards:
