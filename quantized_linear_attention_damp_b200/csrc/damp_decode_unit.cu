@@ -19,20 +19,26 @@
 // then the top three levels over the 8 warps.
 //
 // Per-row operands are gathered once per unit into a small table per warp
-// (k, q, beta*k, the row scale, the row's offset in the block, the KDA
-// decay), by half of the warp's lanes, one row each.
+// (k, q, beta*k, the row scale, the dequantization offset, the row's offset
+// in the block, the KDA decay), by half of the warp's lanes, one row each.
+// A row's load and decode, and its store, are inline PTX with a branch on
+// the row's format marked bra.uni: the format is the same in every lane, so
+// the branch needs no reconvergence.
 //
 // Two CTAs share an SM whenever three stages fit in half of its shared
 // memory (4 stages at 27 FP16 rows): their barriers are independent, so one
-// CTA's arithmetic fills the other's barrier waits.  While columns are
-// combined, warp 6 writes back the previous unit's block (one bulk store,
-// once the barrier after the first half of the step has ordered every
-// writer's fenced rows before it) and warp 7 refills the pipeline
-// (cp.async.bulk of the block, q, k, v, the KDA decays and the head's row
-// directory into a shared-memory ring of stages completing on mbarriers; no
-// tensor map, no multicast).  A named barrier between the two lets the refill
-// start as soon as the stage's old store has read it.  An item needs two CTA
-// barriers.
+// CTA's arithmetic fills the other's barrier waits.  An item needs one CTA
+// barrier: after it, every warp combines the 8 warps' partial sums for its
+// own lanes' columns (the same values in every warp, so no second barrier;
+// the partials are double-buffered by item parity, so a warp that starts
+// the next item cannot overwrite them while another still reads them).
+// Meanwhile warp 6 writes back the previous unit's block (one bulk store,
+// once the barrier has ordered every writer's fenced rows before it) and
+// warp 7 refills the pipeline (cp.async.bulk of the block, q, k, v, the KDA
+// decays and the head's row directory into a shared-memory ring of stages
+// completing on mbarriers; no tensor map, no multicast).  A named barrier
+// between the two lets the refill start as soon as the stage's old store has
+// read it.
 
 #include <cuda_runtime.h>
 
@@ -70,6 +76,7 @@ struct RowTab {
     float4 bs[kPP];      // {b_2p, b_2p+1, s_2p, s_2p+1}: b = beta*k; s = row scale (1 for FP16 rows)
     uint2 off[kPP];      // byte offsets of rows 2p, 2p+1 in the block
     float2 al[kPP];      // KDA decays of rows 2p, 2p+1
+    float2 bz[kPP];      // dequantization offsets of rows 2p, 2p+1: -(2^23+128) byte rows, -0 FP16 rows
     uint32_t soff[kRW];  // byte offset of each byte row's scale in the block
     float amax[kRW];     // row maxima of |X| (byte rows)
     float inv[kRW];      // Q / amax (byte rows; 0 for zero rows)
@@ -120,6 +127,59 @@ __device__ __forceinline__ void byte_row_raw(uint32_t w, float (&f)[4]) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) f[c] = i8_biased(wb, c);
     }
+}
+
+// Four values of one row (this lane's columns), with a uniform branch on the
+// row's format: FP16 row -> the exact values (8 bytes at a8); byte row -> the
+// four INT8 codes at a4 as 2^23 + 128 + code.
+__device__ __forceinline__ void row_load_uni(uint32_t is16, uint32_t a4, uint32_t a8, float (&f)[4]) {
+    asm volatile("{\n\t"
+        ".reg .pred p;\n\t"
+        ".reg .b32 w0, w1, wb;\n\t"
+        ".reg .b16 h0, h1, h2, h3;\n\t"
+        "setp.ne.u32 p, %4, 0;\n\t"
+        "@p bra.uni LF16;\n\t"
+        "ld.shared.u32 w0, [%5];\n\t"
+        "xor.b32 wb, w0, 0x80808080;\n\t"
+        "prmt.b32 %0, wb, %7, 0x7440;\n\t"
+        "prmt.b32 %1, wb, %7, 0x7441;\n\t"
+        "prmt.b32 %2, wb, %7, 0x7442;\n\t"
+        "prmt.b32 %3, wb, %7, 0x7443;\n\t"
+        "bra.uni LEND;\n\t"
+        "LF16:\n\t"
+        "ld.shared.v2.u32 {w0, w1}, [%6];\n\t"
+        "mov.b32 {h0, h1}, w0;\n\t"
+        "mov.b32 {h2, h3}, w1;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t"
+        "cvt.f32.f16 %2, h2;\n\t"
+        "cvt.f32.f16 %3, h3;\n\t"
+        "LEND:\n\t"
+        "}"
+        : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
+        : "r"(is16), "r"(a4), "r"(a8), "r"(0x4B000000u)
+        : "memory");
+}
+
+// Store one row: FP16 row -> the four values rounded to binary16 at a8; byte
+// row -> the code word at a4.  Uniform branch on the format.
+__device__ __forceinline__ void row_store_uni(uint32_t is16, uint32_t a4, uint32_t a8, uint32_t codes,
+                                              float v0, float v1, float v2, float v3) {
+    asm volatile("{\n\t"
+        ".reg .pred p;\n\t"
+        ".reg .b32 h01, h23;\n\t"
+        "setp.ne.u32 p, %0, 0;\n\t"
+        "@p bra.uni SF16;\n\t"
+        "st.shared.u32 [%1], %3;\n\t"
+        "bra.uni SEND;\n\t"
+        "SF16:\n\t"
+        "cvt.rn.f16x2.f32 h01, %5, %4;\n\t"
+        "cvt.rn.f16x2.f32 h23, %7, %6;\n\t"
+        "st.shared.v2.u32 [%2], {h01, h23};\n\t"
+        "SEND:\n\t"
+        "}"
+        :: "r"(is16), "r"(a4), "r"(a8), "r"(codes), "f"(v0), "f"(v1), "f"(v2), "f"(v3)
+        : "memory");
 }
 
 // max |v| over 4 values
@@ -292,10 +352,11 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
 
     // ---- consumers: warp w owns rows [16w, 16w + 16), lane l columns [4l, 4l + 4)
     uint8_t* scratch = smem + a.scratch_off;
-    float* red_u = reinterpret_cast<float*>(scratch);   // [8][128], by warp
-    float* red_w = red_u + kNW * kPD;                   // [8][128], by warp
-    float2* delta2 = reinterpret_cast<float2*>(red_w + kNW * kPD);   // [128] (delta_j, delta_j)
-    float* cpart_s = reinterpret_cast<float*>(delta2 + kPD);        // [8], by warp (16 B padded)
+    float* red_u = reinterpret_cast<float*>(scratch);   // [2][8][128], by warp
+    // per-warp partial sums, double-buffered by item parity: a warp may start
+    // the next item while others still read this item's partials
+    float* red_w = red_u + 2 * kNW * kPD;               // [2][8][128], by warp
+    float* cpart_s = red_w + 2 * kNW * kPD;             // [2][8], by warp
     RowTab* tab = reinterpret_cast<RowTab*>(cpart_s + 16) + warp;
     const int row0 = warp * kRW;
 
@@ -340,6 +401,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     bs[j] = br;
                     bs[2 + j] = sr;
                     reinterpret_cast<uint32_t*>(&tab->off[p])[j] = dir_row(e);
+                    reinterpret_cast<float*>(&tab->bz[p])[j] = f16 ? -0.0f : -8388736.0f;
                     if constexpr (KDA)
                         reinterpret_cast<float*>(&tab->al[p])[j] =
                             reinterpret_cast<const float*>(st + a.st_alpha)[r];
@@ -350,7 +412,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 // c = q^T (beta k) over this warp's rows (any order)
 #pragma unroll
                 for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
-                if (lane == 0) cpart_s[warp] = cp;
+                if (lane == 0) cpart_s[(it & 1) * kNW + warp] = cp;
                 __syncwarp();
             }
             // ---- step 1 (reconstruct) and step 2 (first half), pair by pair:
@@ -368,7 +430,16 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const uint2 o = tab->off[p];
                 const float4 bs = tab->bs[p];
                 const float2 sp = make_float2(bs.z, bs.w);
-                if (fm == 0u) {
+                if constexpr (!FP8) {
+                    float e[4], d[4];
+                    const uint32_t s4 = smem_u32(b4), s8 = smem_u32(b8);
+                    row_load_uni(fm & 1u, s4 + o.x, s8 + o.x, e);
+                    row_load_uni(fm & 2u, s4 + o.y, s8 + o.y, d);
+                    const float2 bz = tab->bz[p];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        x[p][c] = __fmul2_rn(__fadd2_rn(make_float2(e[c], d[c]), bz), sp);
+                } else if (fm == 0u) {
                     float e[4], d[4];
                     byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
                     byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
@@ -432,9 +503,9 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     usum[1] = v[1];
                 }
             }
-            reinterpret_cast<float4*>(red_u + warp * kPD)[lane] =
+            reinterpret_cast<float4*>(red_u + ((it & 1) * kNW + warp) * kPD)[lane] =
                 make_float4(usum[0].x, usum[0].y, usum[1].x, usum[1].y);
-            reinterpret_cast<float4*>(red_w + warp * kPD)[lane] =
+            reinterpret_cast<float4*>(red_w + ((it & 1) * kNW + warp) * kPD)[lane] =
                 make_float4(__fadd_rn(wacc[0].x, wacc[0].y), __fadd_rn(wacc[1].x, wacc[1].y),
                             __fadd_rn(wacc[2].x, wacc[2].y), __fadd_rn(wacc[3].x, wacc[3].y));
         }
@@ -459,62 +530,81 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 issued = it + ahead + 1;
             }
         }
-        // ---- step 2 (second half) + step 3: delta_j and out_j, 128 columns
+        // ---- step 2 (second half) + step 3, in every warp for its lanes'
+        // columns 4l .. 4l+3: u by the top three pairwise levels over the 8
+        // warps' partials, delta = v - u; w, c; warp 0 writes out.  Every warp
+        // reads the same partials, so no second CTA barrier is needed.
         bool bad = false;   // a non-finite input (checked when a.validate)
-        if (tid < kPD) {
-            const int j = tid;
-            if (meta.active == 1) {
-                if (a.validate) {
-                    const float aj = KDA ? reinterpret_cast<const float*>(st + a.st_alpha)[j] : meta.alpha;
-                    bad = !(isfinite(in_at<BF16>(sq, j)) && isfinite(in_at<BF16>(sk, j)) &&
-                            isfinite(in_at<BF16>(st + a.st_v, j)) && isfinite(aj) &&
-                            isfinite(meta.beta));
-                }
-                const float* c0 = red_u + j;
-                const float uj = __fadd_rn(
-                    __fadd_rn(__fadd_rn(c0[0 * kPD], c0[1 * kPD]), __fadd_rn(c0[2 * kPD], c0[3 * kPD])),
-                    __fadd_rn(__fadd_rn(c0[4 * kPD], c0[5 * kPD]), __fadd_rn(c0[6 * kPD], c0[7 * kPD])));
-                const float* w0 = red_w + j;
-                float wj = 0.f;
+        float2 dl[4];
+        if (meta.active == 1) {
+            const float* ru = red_u + (it & 1) * kNW * kPD;
+            const float* rw = red_w + (it & 1) * kNW * kPD;
+            float2 u01[2][4];   // [column pair][tree node]
 #pragma unroll
-                for (int q2 = 0; q2 < kNW; ++q2) wj = __fadd_rn(wj, w0[q2 * kPD]);
-                const float4 c4a = reinterpret_cast<const float4*>(cpart_s)[0];
-                const float4 c4b = reinterpret_cast<const float4*>(cpart_s)[1];
-                const float c = ((c4a.x + c4a.y) + (c4a.z + c4a.w)) + ((c4b.x + c4b.y) + (c4b.z + c4b.w));
-                const float vj = in_at<BF16>(st + a.st_v, j);
-                const float dj = __fsub_rn(vj, uj);
-                delta2[j] = f2(dj);
-                a.out[(size_t)meta.unit * kPD + j] = __fmaf_rn(c, dj, wj);
-            } else if (meta.unit >= 0) {
-                a.out[(size_t)meta.unit * kPD + j] = 0.f;
-                if (j == 0 && meta.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float4 a0 = reinterpret_cast<const float4*>(ru + (2 * q2) * kPD)[lane];
+                const float4 a1 = reinterpret_cast<const float4*>(ru + (2 * q2 + 1) * kPD)[lane];
+                u01[0][q2] = __fadd2_rn(make_float2(a0.x, a0.y), make_float2(a1.x, a1.y));
+                u01[1][q2] = __fadd2_rn(make_float2(a0.z, a0.w), make_float2(a1.z, a1.w));
             }
-        }
-        if (a.validate) {
-            bad = __syncthreads_or(bad);
-            if (bad) {
-                // the unit is skipped: out row zeroed, block neither updated nor stored
-                if (tid < kPD) a.out[(size_t)meta.unit * kPD + tid] = 0.f;
-                if (tid == 0) {
-                    reinterpret_cast<PMeta*>(st + a.st_meta)->active = 0;
-                    atomicOr(a.status, DAMP_EFLAG_NONFINITE);
+            float2 uu[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                uu[h] = __fadd2_rn(__fadd2_rn(u01[h][0], u01[h][1]), __fadd2_rn(u01[h][2], u01[h][3]));
+            float2 ww[2] = {f2(0.f), f2(0.f)};
+#pragma unroll
+            for (int q2 = 0; q2 < kNW; ++q2) {
+                const float4 b0 = reinterpret_cast<const float4*>(rw + q2 * kPD)[lane];
+                ww[0] = __fadd2_rn(ww[0], make_float2(b0.x, b0.y));
+                ww[1] = __fadd2_rn(ww[1], make_float2(b0.z, b0.w));
+            }
+            const float4 c4a = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[0];
+            const float4 c4b = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[1];
+            const float c = ((c4a.x + c4a.y) + (c4a.z + c4a.w)) + ((c4b.x + c4b.y) + (c4b.z + c4b.w));
+            float vv[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) vv[cc] = in_at<BF16>(st + a.st_v, 4 * lane + cc);
+            // delta = fl(v - u) (the negation is exact)
+            const float2 d01 = __fadd2_rn(make_float2(vv[0], vv[1]), make_float2(-uu[0].x, -uu[0].y));
+            const float2 d23 = __fadd2_rn(make_float2(vv[2], vv[3]), make_float2(-uu[1].x, -uu[1].y));
+            dl[0] = f2(d01.x);
+            dl[1] = f2(d01.y);
+            dl[2] = f2(d23.x);
+            dl[3] = f2(d23.y);
+            if (warp == 0) {
+                const float2 o01 = __ffma2_rn(f2(c), d01, ww[0]);
+                const float2 o23 = __ffma2_rn(f2(c), d23, ww[1]);
+                reinterpret_cast<float4*>(a.out + (size_t)meta.unit * kPD)[lane] =
+                    make_float4(o01.x, o01.y, o23.x, o23.y);
+            }
+            if (a.validate) {
+                // every warp checks the same inputs: the vote is uniform over the CTA
+                bool f = isfinite(meta.beta) && isfinite(meta.alpha);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int j = 4 * lane + cc;
+                    f = f && isfinite(vv[cc]) && isfinite(in_at<BF16>(sq, j)) && isfinite(in_at<BF16>(sk, j));
+                    if constexpr (KDA) f = f && isfinite(reinterpret_cast<const float*>(st + a.st_alpha)[j]);
+                }
+                bad = __any_sync(0xffffffffu, !f);
+                if (bad) {
+                    // the unit is skipped: out row zeroed, block neither updated nor stored
+                    if (warp == 0) reinterpret_cast<float4*>(a.out + (size_t)meta.unit * kPD)[lane] =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (tid == 0) {
+                        reinterpret_cast<PMeta*>(st + a.st_meta)->active = 0;
+                        atomicOr(a.status, DAMP_EFLAG_NONFINITE);
+                    }
                 }
             }
-        } else {
-            __syncthreads();
+        } else if (meta.unit >= 0 && warp == 0) {
+            reinterpret_cast<float4*>(a.out + (size_t)meta.unit * kPD)[lane] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lane == 0 && meta.active < 0) atomicOr(a.status, DAMP_EFLAG_SLOT_RANGE);
         }
 
         // ---- step 2 (update) + step 6: X = S' + b delta^T, requantize in place
         if (any && !bad) {
-            float2 dl[4];
-            {
-                const float4 d0 = reinterpret_cast<const float4*>(delta2 + 4 * lane)[0];
-                const float4 d1 = reinterpret_cast<const float4*>(delta2 + 4 * lane)[1];
-                dl[0] = make_float2(d0.x, d0.y);
-                dl[1] = make_float2(d0.z, d0.w);
-                dl[2] = make_float2(d1.x, d1.y);
-                dl[3] = make_float2(d1.z, d1.w);
-            }
             float am[kRW];
 #pragma unroll
             for (int p = 0; p < kPP; ++p) {
@@ -523,13 +613,11 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const float2 bp = make_float2(bs.x, bs.y);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) x[p][c] = __ffma2_rn(bp, dl[c], x[p][c]);
-                am[2 * p] = am[2 * p + 1] = 0.f;
-                if (!(fm & 1u))
-                    am[2 * p] = __uint_as_float(__reduce_max_sync(
-                        0xffffffffu, __float_as_uint(absmax4v(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x))));
-                if (!(fm & 2u))
-                    am[2 * p + 1] = __uint_as_float(__reduce_max_sync(
-                        0xffffffffu, __float_as_uint(absmax4v(x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y))));
+                (void)fm;
+                am[2 * p] = __uint_as_float(__reduce_max_sync(
+                    0xffffffffu, __float_as_uint(absmax4v(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x))));
+                am[2 * p + 1] = __uint_as_float(__reduce_max_sync(
+                    0xffffffffu, __float_as_uint(absmax4v(x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y))));
             }
             if (lane == 0) {
 #pragma unroll
@@ -537,19 +625,36 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     *reinterpret_cast<float4*>(&tab->amax[i]) = make_float4(am[i], am[i + 1], am[i + 2], am[i + 3]);
             }
             __syncwarp();
-            // per byte row r = lane & 15: lanes 0-15 form inv = fl(Q/a), lanes
-            // 16-31 scale = fl(a/Q) and store it into the block
+            // per byte row r = lane & 15: inv = fl(Q/a) into the table (lanes
+            // 0-15), scale = fl(a/Q) into the block (lanes 16-31)
             {
                 const int r = lane & 15;
                 const bool byte_row = !((m16 >> r) & 1u);
                 const float am_r = tab->amax[r];
-                float res = 0.f;
-                if (byte_row) res = lane < 16 ? __fdiv_rn(kQ, am_r) : __fdiv_rn(am_r, kQ);
-                const float inv_r = __shfl_sync(0xffffffffu, res, r);
-                if (byte_row) {
-                    const bool zero = am_r == 0.0f || isinf(inv_r);
-                    if (lane < 16) tab->inv[r] = zero ? 0.0f : res;
-                    else *reinterpret_cast<float*>(blk + tab->soff[r]) = zero ? 0.0f : res;
+                if constexpr (FP8) {
+                    float res = 0.f;
+                    if (byte_row) res = lane < 16 ? __fdiv_rn(kQ, am_r) : __fdiv_rn(am_r, kQ);
+                    const float inv_r = __shfl_sync(0xffffffffu, res, r);
+                    if (byte_row) {
+                        const bool zero = am_r == 0.0f || isinf(inv_r);
+                        if (lane < 16) tab->inv[r] = zero ? 0.0f : res;
+                        else *reinterpret_cast<float*>(blk + tab->soff[r]) = zero ? 0.0f : res;
+                    }
+                } else {
+                    // every lane forms both: inv by IEEE division, scale by
+                    // division by the constant 127 (Markstein: one product and
+                    // two fused corrections give the correctly rounded
+                    // quotient for every finite a >= 0; a = inf is kept)
+                    const float inv = __fdiv_rn(127.0f, am_r);
+                    const float y = 0.007874015718698501587f;   // RN(1/127)
+                    const float q0 = __fmul_rn(am_r, y);
+                    const float q1 = __fmaf_rn(__fmaf_rn(-q0, 127.0f, am_r), y, q0);
+                    const float scale = isinf(am_r) ? am_r : q1;
+                    if (byte_row) {
+                        const bool zero = am_r == 0.0f || isinf(inv);
+                        if (lane < 16) tab->inv[r] = zero ? 0.0f : inv;
+                        else *reinterpret_cast<float*>(blk + tab->soff[r]) = zero ? 0.0f : scale;
+                    }
                 }
             }
             __syncwarp();
@@ -558,7 +663,12 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const uint32_t fm = (m16 >> (2 * p)) & 3u;
                 const uint2 o = tab->off[p];
                 const float2 ip = *reinterpret_cast<const float2*>(&tab->inv[2 * p]);
-                if (fm == 0u) {
+                if constexpr (!FP8) {
+                    const uint2 cw = quant_pair4<false>(x[p], ip);
+                    const uint32_t s4 = smem_u32(b4), s8 = smem_u32(b8);
+                    row_store_uni(fm & 1u, s4 + o.x, s8 + o.x, cw.x, x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x);
+                    row_store_uni(fm & 2u, s4 + o.y, s8 + o.y, cw.y, x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y);
+                } else if (fm == 0u) {
                     const uint2 cw = quant_pair4<FP8>(x[p], ip);
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) = cw.x;
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) = cw.y;
@@ -634,7 +744,7 @@ uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
     off += sizeof(PMeta);
     a.stage_bytes = up(off, 128);
     const uint32_t scratch =
-        up((2 * kNW * kPD + 2 * kPD + 16) * 4 + kNW * (uint32_t)sizeof(RowTab), 128);
+        up((4 * kNW * kPD + 16) * 4 + kNW * (uint32_t)sizeof(RowTab), 128);
     uint32_t ns = (budget - scratch - 128) / a.stage_bytes;
     if (ns > 6) ns = 6;
     if (ns < 3) return 0;
