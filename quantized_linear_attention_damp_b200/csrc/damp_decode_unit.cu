@@ -21,9 +21,11 @@
 // Per-row operands are gathered once per unit into a small table per warp
 // (k, q, beta*k, the row scale, the dequantization offset, the row's offset
 // in the block, the KDA decay), by half of the warp's lanes, one row each.
-// A row's load and decode, and its store, are inline PTX with a branch on
-// the row's format marked bra.uni: the format is the same in every lane, so
-// the branch needs no reconvergence.
+// A row's words are loaded from wherever its format keeps them, outside any
+// branch, so that the loads of later rows can be issued ahead; the decode,
+// and later the store, are inline PTX with a branch on the row's format
+// marked bra.uni: the format is the same in every lane, so the branch needs
+// no reconvergence.  A pair of byte rows is stored behind one test.
 //
 // Two CTAs share an SM whenever three stages fit in half of its shared
 // memory (4 stages at 27 FP16 rows): their barriers are independent, so one
@@ -129,56 +131,126 @@ __device__ __forceinline__ void byte_row_raw(uint32_t w, float (&f)[4]) {
     }
 }
 
-// Four values of one row (this lane's columns), with a uniform branch on the
-// row's format: FP16 row -> the exact values (8 bytes at a8); byte row -> the
-// four INT8 codes at a4 as 2^23 + 128 + code.
-__device__ __forceinline__ void row_load_uni(uint32_t is16, uint32_t a4, uint32_t a8, float (&f)[4]) {
-    asm volatile("{\n\t"
-        ".reg .pred p;\n\t"
-        ".reg .b32 w0, w1, wb;\n\t"
-        ".reg .b16 h0, h1, h2, h3;\n\t"
-        "setp.ne.u32 p, %4, 0;\n\t"
-        "@p bra.uni LF16;\n\t"
-        "ld.shared.u32 w0, [%5];\n\t"
-        "xor.b32 wb, w0, 0x80808080;\n\t"
-        "prmt.b32 %0, wb, %7, 0x7440;\n\t"
-        "prmt.b32 %1, wb, %7, 0x7441;\n\t"
-        "prmt.b32 %2, wb, %7, 0x7442;\n\t"
-        "prmt.b32 %3, wb, %7, 0x7443;\n\t"
-        "bra.uni LEND;\n\t"
-        "LF16:\n\t"
-        "ld.shared.v2.u32 {w0, w1}, [%6];\n\t"
-        "mov.b32 {h0, h1}, w0;\n\t"
-        "mov.b32 {h2, h3}, w1;\n\t"
-        "cvt.f32.f16 %0, h0;\n\t"
-        "cvt.f32.f16 %1, h1;\n\t"
-        "cvt.f32.f16 %2, h2;\n\t"
-        "cvt.f32.f16 %3, h3;\n\t"
-        "LEND:\n\t"
-        "}"
-        : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
-        : "r"(is16), "r"(a4), "r"(a8), "r"(0x4B000000u)
-        : "memory");
+// A float2 held in one 64-bit register (the operand type of the packed FP32
+// instructions) and back.
+__device__ __forceinline__ float2 as_f2(unsigned long long v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ unsigned long long as_u64(float2 v) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+    return r;
 }
 
-// Store one row: FP16 row -> the four values rounded to binary16 at a8; byte
-// row -> the code word at a4.  Uniform branch on the format.
-__device__ __forceinline__ void row_store_uni(uint32_t is16, uint32_t a4, uint32_t a8, uint32_t codes,
-                                              float v0, float v1, float v2, float v3) {
-    asm volatile("{\n\t"
-        ".reg .pred p;\n\t"
-        ".reg .b32 h01, h23;\n\t"
-        "setp.ne.u32 p, %0, 0;\n\t"
-        "@p bra.uni SF16;\n\t"
-        "st.shared.u32 [%1], %3;\n\t"
-        "bra.uni SEND;\n\t"
-        "SF16:\n\t"
-        "cvt.rn.f16x2.f32 h01, %5, %4;\n\t"
-        "cvt.rn.f16x2.f32 h23, %7, %6;\n\t"
-        "st.shared.v2.u32 [%2], {h01, h23};\n\t"
-        "SEND:\n\t"
+// Both rows of a pair decoded and dequantized from their words, which the
+// caller has loaded (rows 2p, 2p + 1 as .x, .y; FP16 flags = bits 2p and
+// 2p + 1 of m): x[c] = fl((raw_c + bz) * s), raw = the exact binary16 value
+// (FP16 row: both words) or 2^23 + 128 + code (byte row: the codes in the
+// first word).  Each row's format is a uniform branch (bra.uni: the same in
+// every lane); the offset and the scale are packed operations on the pair.
+__device__ __forceinline__ void pair_decode(int P, uint32_t m, uint32_t we0, uint32_t we1,
+                                                uint32_t wo0, uint32_t wo1, float2 bz, float2 sp,
+                                                float2 (&x)[4]) {
+    unsigned long long r0, r1, r2, r3;
+    asm("{\n\t"
+        ".reg .pred p, pe, po;\n\t"
+        ".reg .b32 t, wb, e0, e1, e2, e3, d0, d1, d2, d3;\n\t"
+        ".reg .b16 h0, h1, h2, h3;\n\t"
+        "and.b32 t, %4, %10;\n\t"
+        "setp.ne.u32 pe, t, 0;\n\t"
+        "@pe bra.uni EF16;\n\t"
+        "xor.b32 wb, %5, 0x80808080;\n\t"
+        "prmt.b32 e0, wb, %9, 0x7440;\n\t"
+        "prmt.b32 e1, wb, %9, 0x7441;\n\t"
+        "prmt.b32 e2, wb, %9, 0x7442;\n\t"
+        "prmt.b32 e3, wb, %9, 0x7443;\n\t"
+        "bra.uni EEND;\n\t"
+        "EF16:\n\t"
+        "mov.b32 {h0, h1}, %5;\n\t"
+        "mov.b32 {h2, h3}, %6;\n\t"
+        "cvt.f32.f16 e0, h0;\n\t"
+        "cvt.f32.f16 e1, h1;\n\t"
+        "cvt.f32.f16 e2, h2;\n\t"
+        "cvt.f32.f16 e3, h3;\n\t"
+        "EEND:\n\t"
+        "and.b32 t, %4, %11;\n\t"
+        "setp.ne.u32 po, t, 0;\n\t"
+        "@po bra.uni OF16;\n\t"
+        "xor.b32 wb, %7, 0x80808080;\n\t"
+        "prmt.b32 d0, wb, %9, 0x7440;\n\t"
+        "prmt.b32 d1, wb, %9, 0x7441;\n\t"
+        "prmt.b32 d2, wb, %9, 0x7442;\n\t"
+        "prmt.b32 d3, wb, %9, 0x7443;\n\t"
+        "bra.uni PEND;\n\t"
+        "OF16:\n\t"
+        "mov.b32 {h0, h1}, %7;\n\t"
+        "mov.b32 {h2, h3}, %8;\n\t"
+        "cvt.f32.f16 d0, h0;\n\t"
+        "cvt.f32.f16 d1, h1;\n\t"
+        "cvt.f32.f16 d2, h2;\n\t"
+        "cvt.f32.f16 d3, h3;\n\t"
+        "PEND:\n\t"
+        "mov.b64 %0, {e0, d0};\n\t"
+        "mov.b64 %1, {e1, d1};\n\t"
+        "mov.b64 %2, {e2, d2};\n\t"
+        "mov.b64 %3, {e3, d3};\n\t"
+        "add.rn.f32x2 %0, %0, %12;\n\t"
+        "add.rn.f32x2 %1, %1, %12;\n\t"
+        "add.rn.f32x2 %2, %2, %12;\n\t"
+        "add.rn.f32x2 %3, %3, %12;\n\t"
+        "mul.rn.f32x2 %0, %0, %13;\n\t"
+        "mul.rn.f32x2 %1, %1, %13;\n\t"
+        "mul.rn.f32x2 %2, %2, %13;\n\t"
+        "mul.rn.f32x2 %3, %3, %13;\n\t"
         "}"
-        :: "r"(is16), "r"(a4), "r"(a8), "r"(codes), "f"(v0), "f"(v1), "f"(v2), "f"(v3)
+        : "=l"(r0), "=l"(r1), "=l"(r2), "=l"(r3)
+        : "r"(m), "r"(we0), "r"(we1), "r"(wo0), "r"(wo1), "r"(0x4B000000u),
+          "r"(1u << (2 * P)), "r"(2u << (2 * P)), "l"(as_u64(bz)), "l"(as_u64(sp)));
+    x[0] = as_f2(r0); x[1] = as_f2(r1); x[2] = as_f2(r2); x[3] = as_f2(r3);
+}
+
+// Store both rows of a pair: the two code words when both are byte rows (one
+// uniform test), else row by row (FP16 row -> its four values rounded to
+// binary16; byte row -> its code word).
+__device__ __forceinline__ void pair_store(int P, uint32_t m, uint32_t a4e, uint32_t a8e, uint32_t a4o,
+                                               uint32_t a8o, uint2 cw, const float2 (&x)[4]) {
+    asm volatile("{\n\t"
+        ".reg .pred p, pe, po;\n\t"
+        ".reg .b32 t, h01, h23;\n\t"
+        "and.b32 t, %0, %15;\n\t"
+        "setp.ne.u32 p, t, 0;\n\t"
+        "@p bra.uni QMIX;\n\t"
+        "st.shared.u32 [%1], %5;\n\t"
+        "st.shared.u32 [%3], %6;\n\t"
+        "bra.uni QEND;\n\t"
+        "QMIX:\n\t"
+        "and.b32 t, %0, %16;\n\t"
+        "setp.ne.u32 pe, t, 0;\n\t"
+        "@pe bra.uni QEF;\n\t"
+        "st.shared.u32 [%1], %5;\n\t"
+        "bra.uni QEE;\n\t"
+        "QEF:\n\t"
+        "cvt.rn.f16x2.f32 h01, %8, %7;\n\t"
+        "cvt.rn.f16x2.f32 h23, %10, %9;\n\t"
+        "st.shared.v2.u32 [%2], {h01, h23};\n\t"
+        "QEE:\n\t"
+        "and.b32 t, %0, %17;\n\t"
+        "setp.ne.u32 po, t, 0;\n\t"
+        "@po bra.uni QOF;\n\t"
+        "st.shared.u32 [%3], %6;\n\t"
+        "bra.uni QEND;\n\t"
+        "QOF:\n\t"
+        "cvt.rn.f16x2.f32 h01, %12, %11;\n\t"
+        "cvt.rn.f16x2.f32 h23, %14, %13;\n\t"
+        "st.shared.v2.u32 [%4], {h01, h23};\n\t"
+        "QEND:\n\t"
+        "}"
+        :: "r"(m), "r"(a4e), "r"(a8e), "r"(a4o), "r"(a8o), "r"(cw.x), "r"(cw.y),
+           "f"(x[0].x), "f"(x[1].x), "f"(x[2].x), "f"(x[3].x),
+           "f"(x[0].y), "f"(x[1].y), "f"(x[2].y), "f"(x[3].y),
+           "r"(3u << (2 * P)), "r"(1u << (2 * P)), "r"(2u << (2 * P))
         : "memory");
 }
 
@@ -431,14 +503,13 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const float4 bs = tab->bs[p];
                 const float2 sp = make_float2(bs.z, bs.w);
                 if constexpr (!FP8) {
-                    float e[4], d[4];
-                    const uint32_t s4 = smem_u32(b4), s8 = smem_u32(b8);
-                    row_load_uni(fm & 1u, s4 + o.x, s8 + o.x, e);
-                    row_load_uni(fm & 2u, s4 + o.y, s8 + o.y, d);
-                    const float2 bz = tab->bz[p];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        x[p][c] = __fmul2_rn(__fadd2_rn(make_float2(e[c], d[c]), bz), sp);
+                    // each row's words wherever its format keeps them (a byte
+                    // row reads one word more than it uses, inside the stage),
+                    // loaded outside the format branches so that they can be
+                    // issued ahead; then the decode
+                    const uint32_t* pe = reinterpret_cast<const uint32_t*>((fm & 1u) ? b8 + o.x : b4 + o.x);
+                    const uint32_t* po = reinterpret_cast<const uint32_t*>((fm & 2u) ? b8 + o.y : b4 + o.y);
+                    pair_decode(p, m16, pe[0], pe[1], po[0], po[1], tab->bz[p], sp, x[p]);
                 } else if (fm == 0u) {
                     float e[4], d[4];
                     byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
@@ -551,16 +622,6 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
 #pragma unroll
             for (int h = 0; h < 2; ++h)
                 uu[h] = __fadd2_rn(__fadd2_rn(u01[h][0], u01[h][1]), __fadd2_rn(u01[h][2], u01[h][3]));
-            float2 ww[2] = {f2(0.f), f2(0.f)};
-#pragma unroll
-            for (int q2 = 0; q2 < kNW; ++q2) {
-                const float4 b0 = reinterpret_cast<const float4*>(rw + q2 * kPD)[lane];
-                ww[0] = __fadd2_rn(ww[0], make_float2(b0.x, b0.y));
-                ww[1] = __fadd2_rn(ww[1], make_float2(b0.z, b0.w));
-            }
-            const float4 c4a = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[0];
-            const float4 c4b = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[1];
-            const float c = ((c4a.x + c4a.y) + (c4a.z + c4a.w)) + ((c4b.x + c4b.y) + (c4b.z + c4b.w));
             float vv[4];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) vv[cc] = in_at<BF16>(st + a.st_v, 4 * lane + cc);
@@ -572,6 +633,17 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             dl[2] = f2(d23.x);
             dl[3] = f2(d23.y);
             if (warp == 0) {
+                // out = w + c delta (only this warp needs w and c)
+                float2 ww[2] = {f2(0.f), f2(0.f)};
+#pragma unroll
+                for (int q2 = 0; q2 < kNW; ++q2) {
+                    const float4 b0 = reinterpret_cast<const float4*>(rw + q2 * kPD)[lane];
+                    ww[0] = __fadd2_rn(ww[0], make_float2(b0.x, b0.y));
+                    ww[1] = __fadd2_rn(ww[1], make_float2(b0.z, b0.w));
+                }
+                const float4 c4a = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[0];
+                const float4 c4b = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[1];
+                const float c = ((c4a.x + c4a.y) + (c4a.z + c4a.w)) + ((c4b.x + c4b.y) + (c4b.z + c4b.w));
                 const float2 o01 = __ffma2_rn(f2(c), d01, ww[0]);
                 const float2 o23 = __ffma2_rn(f2(c), d23, ww[1]);
                 reinterpret_cast<float4*>(a.out + (size_t)meta.unit * kPD)[lane] =
@@ -666,8 +738,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 if constexpr (!FP8) {
                     const uint2 cw = quant_pair4<false>(x[p], ip);
                     const uint32_t s4 = smem_u32(b4), s8 = smem_u32(b8);
-                    row_store_uni(fm & 1u, s4 + o.x, s8 + o.x, cw.x, x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x);
-                    row_store_uni(fm & 2u, s4 + o.y, s8 + o.y, cw.y, x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y);
+                    pair_store(p, m16, s4 + o.x, s8 + o.x, s4 + o.y, s8 + o.y, cw, x[p]);
                 } else if (fm == 0u) {
                     const uint2 cw = quant_pair4<FP8>(x[p], ip);
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) = cw.x;
