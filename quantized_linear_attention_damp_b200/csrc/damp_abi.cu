@@ -587,7 +587,8 @@ int damp_block_to_logical(const damp_pool* pool, int h, const void* block, float
     for (int i = 0; i < DK; ++i) {
         if (is_fp16_row(d, h, i)) {
             scale[i] = 0.0f;
-            memcpy(half + (size_t)i * DV, b + f16_off + (size_t)r16 * 2 * DV, (size_t)2 * DV);
+            const uint8_t* row = b + f16_off + (size_t)r16 * 2 * DV;
+            for (int j = 0; j < DV; ++j) memcpy(half + (size_t)i * DV + j, row + damp::f16_pos(j, DV), 2);
             memset(code + (size_t)i * DV, 0, DV);
             ++r16;
         } else {
@@ -618,7 +619,8 @@ int damp_block_from_logical(const damp_pool* pool, int h, const float* scale,
     int r16 = 0, r8 = 0;
     for (int i = 0; i < DK; ++i) {
         if (is_fp16_row(d, h, i)) {
-            memcpy(b + f16_off + (size_t)r16 * 2 * DV, half + (size_t)i * DV, (size_t)2 * DV);
+            uint8_t* row = b + f16_off + (size_t)r16 * 2 * DV;
+            for (int j = 0; j < DV; ++j) memcpy(row + damp::f16_pos(j, DV), half + (size_t)i * DV + j, 2);
             ++r16;
         } else {
             memcpy(b + (size_t)r8 * 4, &scale[i], 4);

@@ -62,7 +62,7 @@ __device__ __forceinline__ float load_shat(const uint8_t* blk, int codec, uint32
                                            int i, int j, int d_v) {
     if (codec == 0) return reinterpret_cast<const float*>(blk)[(size_t)i * d_v + j];
     const uint8_t* row = blk + dir_row(e);
-    if (e >> 31) return __half2float(reinterpret_cast<const __half*>(row)[j]);
+    if (e >> 31) return __half2float(*reinterpret_cast<const __half*>(row + f16_pos(j, d_v)));
     if (codec == 2) return __fmul_rn(e4m3_value(row[j]), s);
     return __fmul_rn((float)(int8_t)row[j], s);
 }
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kAnyThreads) decode_any_kernel(const StepArgs 
 #pragma unroll
             for (int t = 0; t < kColsPerLane; ++t) {
                 const int j = lane + 32 * t;
-                if (j < d_v) reinterpret_cast<__half*>(row)[j] = __float2half_rn(x[t]);
+                if (j < d_v) *reinterpret_cast<__half*>(row + f16_pos(j, d_v)) = __float2half_rn(x[t]);
             }
             continue;
         }
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kAnyThreads) codec_any_kernel(const CodecArgs 
 #pragma unroll
             for (int t = 0; t < kColsPerLane; ++t) {
                 const int j = lane + 32 * t;
-                if (j < d_v) reinterpret_cast<__half*>(row)[j] = __float2half_rn(x[t]);
+                if (j < d_v) *reinterpret_cast<__half*>(row + f16_pos(j, d_v)) = __float2half_rn(x[t]);
             }
             return;
         }

@@ -211,47 +211,59 @@ __device__ __forceinline__ void pair_decode(int P, uint32_t m, uint32_t we0, uin
     x[0] = as_f2(r0); x[1] = as_f2(r1); x[2] = as_f2(r2); x[3] = as_f2(r3);
 }
 
-// Store both rows of a pair: the two code words when both are byte rows (one
-// uniform test), else row by row (FP16 row -> its four values rounded to
-// binary16; byte row -> its code word).
-__device__ __forceinline__ void pair_store(int P, uint32_t m, uint32_t a4e, uint32_t a8e, uint32_t a4o,
-                                               uint32_t a8o, uint2 cw, const float2 (&x)[4]) {
+// Store both rows of a pair at their words a_e, a_o: the two code words when
+// both are byte rows (one uniform test), else row by row (byte row -> its
+// code word; FP16 row -> its four values rounded to binary16, one word in
+// each plane).
+__device__ __forceinline__ void pair_store(int P, uint32_t m, uint32_t ae, uint32_t ao, uint2 cw,
+                                           const float2 (&x)[4]) {
     asm volatile("{\n\t"
         ".reg .pred p, pe, po;\n\t"
         ".reg .b32 t, h01, h23;\n\t"
-        "and.b32 t, %0, %15;\n\t"
+        "and.b32 t, %0, %13;\n\t"
         "setp.ne.u32 p, t, 0;\n\t"
         "@p bra.uni QMIX;\n\t"
-        "st.shared.u32 [%1], %5;\n\t"
-        "st.shared.u32 [%3], %6;\n\t"
+        "st.shared.u32 [%1], %3;\n\t"
+        "st.shared.u32 [%2], %4;\n\t"
         "bra.uni QEND;\n\t"
         "QMIX:\n\t"
-        "and.b32 t, %0, %16;\n\t"
+        "and.b32 t, %0, %14;\n\t"
         "setp.ne.u32 pe, t, 0;\n\t"
         "@pe bra.uni QEF;\n\t"
-        "st.shared.u32 [%1], %5;\n\t"
+        "st.shared.u32 [%1], %3;\n\t"
         "bra.uni QEE;\n\t"
         "QEF:\n\t"
-        "cvt.rn.f16x2.f32 h01, %8, %7;\n\t"
-        "cvt.rn.f16x2.f32 h23, %10, %9;\n\t"
-        "st.shared.v2.u32 [%2], {h01, h23};\n\t"
+        "cvt.rn.f16x2.f32 h01, %6, %5;\n\t"
+        "cvt.rn.f16x2.f32 h23, %8, %7;\n\t"
+        "st.shared.u32 [%1], h01;\n\t"
+        "st.shared.u32 [%1+128], h23;\n\t"
         "QEE:\n\t"
-        "and.b32 t, %0, %17;\n\t"
+        "and.b32 t, %0, %15;\n\t"
         "setp.ne.u32 po, t, 0;\n\t"
         "@po bra.uni QOF;\n\t"
-        "st.shared.u32 [%3], %6;\n\t"
+        "st.shared.u32 [%2], %4;\n\t"
         "bra.uni QEND;\n\t"
         "QOF:\n\t"
-        "cvt.rn.f16x2.f32 h01, %12, %11;\n\t"
-        "cvt.rn.f16x2.f32 h23, %14, %13;\n\t"
-        "st.shared.v2.u32 [%4], {h01, h23};\n\t"
+        "cvt.rn.f16x2.f32 h01, %10, %9;\n\t"
+        "cvt.rn.f16x2.f32 h23, %12, %11;\n\t"
+        "st.shared.u32 [%2], h01;\n\t"
+        "st.shared.u32 [%2+128], h23;\n\t"
         "QEND:\n\t"
         "}"
-        :: "r"(m), "r"(a4e), "r"(a8e), "r"(a4o), "r"(a8o), "r"(cw.x), "r"(cw.y),
+        :: "r"(m), "r"(ae), "r"(ao), "r"(cw.x), "r"(cw.y),
            "f"(x[0].x), "f"(x[1].x), "f"(x[2].x), "f"(x[3].x),
            "f"(x[0].y), "f"(x[1].y), "f"(x[2].y), "f"(x[3].y),
            "r"(3u << (2 * P)), "r"(1u << (2 * P)), "r"(2u << (2 * P))
         : "memory");
+}
+
+// This lane's two words of an FP16 row (one per plane) and their store.
+__device__ __forceinline__ uint2 f16_words(const uint8_t* w) {
+    return make_uint2(*reinterpret_cast<const uint32_t*>(w), *reinterpret_cast<const uint32_t*>(w + kPD));
+}
+__device__ __forceinline__ void f16_store(const uint8_t* w, uint2 h) {
+    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(w)) = h.x;
+    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(w) + kPD) = h.y;
 }
 
 // max |v| over 4 values
@@ -448,7 +460,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
         const uint8_t* sk = st + a.st_k;
         const uint32_t* sdir = reinterpret_cast<const uint32_t*>(st + a.st_dir);
         const uint8_t* b4 = blk + 4 * lane;   // this lane's 4 codes of a byte row
-        const uint8_t* b8 = blk + 8 * lane;   // this lane's 4 values of an FP16 row
+        // an FP16 row keeps this lane's 4 values as two words, at b4 and at
+        // b4 + 128 (its two planes)
 
         float2 x[kPP][4];
         uint32_t m16 = 0;   // bit i: row row0 + i is an FP16 row
@@ -503,13 +516,14 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const float4 bs = tab->bs[p];
                 const float2 sp = make_float2(bs.z, bs.w);
                 if constexpr (!FP8) {
-                    // each row's words wherever its format keeps them (a byte
-                    // row reads one word more than it uses, inside the stage),
+                    // each row's words (a byte row's word, or an FP16 row's
+                    // two plane words; a byte row also reads the word 128
+                    // bytes on, inside the stage, and does not use it),
                     // loaded outside the format branches so that they can be
                     // issued ahead; then the decode
-                    const uint32_t* pe = reinterpret_cast<const uint32_t*>((fm & 1u) ? b8 + o.x : b4 + o.x);
-                    const uint32_t* po = reinterpret_cast<const uint32_t*>((fm & 2u) ? b8 + o.y : b4 + o.y);
-                    pair_decode(p, m16, pe[0], pe[1], po[0], po[1], tab->bz[p], sp, x[p]);
+                    const uint32_t* pe = reinterpret_cast<const uint32_t*>(b4 + o.x);
+                    const uint32_t* po = reinterpret_cast<const uint32_t*>(b4 + o.y);
+                    pair_decode(p, m16, pe[0], pe[kPD / 4], po[0], po[kPD / 4], tab->bz[p], sp, x[p]);
                 } else if (fm == 0u) {
                     float e[4], d[4];
                     byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
@@ -522,8 +536,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     }
                 } else if (fm == 3u) {
                     float e[4], d[4];
-                    f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.x), e);
-                    f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.y), d);
+                    f16x4_to_f32(f16_words(b4 + o.x), e);
+                    f16x4_to_f32(f16_words(b4 + o.y), d);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) x[p][c] = make_float2(e[c], d[c]);
                 } else {
@@ -531,11 +545,11 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     // -0 and scaled by 1 (both exact, signed zeros kept)
                     float e[4], d[4];
                     if (fm == 1u) {
-                        f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.x), e);
+                        f16x4_to_f32(f16_words(b4 + o.x), e);
                         byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
                     } else {
                         byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
-                        f16x4_to_f32(*reinterpret_cast<const uint2*>(b8 + o.y), d);
+                        f16x4_to_f32(f16_words(b4 + o.y), d);
                     }
                     const float2 bz = fm == 1u ? make_float2(-0.0f, -8388736.0f)
                                                : make_float2(-8388736.0f, -0.0f);
@@ -737,8 +751,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const float2 ip = *reinterpret_cast<const float2*>(&tab->inv[2 * p]);
                 if constexpr (!FP8) {
                     const uint2 cw = quant_pair4<false>(x[p], ip);
-                    const uint32_t s4 = smem_u32(b4), s8 = smem_u32(b8);
-                    pair_store(p, m16, s4 + o.x, s8 + o.x, s4 + o.y, s8 + o.y, cw, x[p]);
+                    const uint32_t s4 = smem_u32(b4);
+                    pair_store(p, m16, s4 + o.x, s4 + o.y, cw, x[p]);
                 } else if (fm == 0u) {
                     const uint2 cw = quant_pair4<FP8>(x[p], ip);
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) = cw.x;
@@ -748,12 +762,12 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                                                   make_float2(x[p][2].x, x[p][3].x));
                     const uint2 ho = quant_fp16x4(make_float2(x[p][0].y, x[p][1].y),
                                                   make_float2(x[p][2].y, x[p][3].y));
-                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.x) = he;
-                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.y) = ho;
+                    f16_store(b4 + o.x, he);
+                    f16_store(b4 + o.y, ho);
                 } else if (fm == 1u) {
                     const uint2 he = quant_fp16x4(make_float2(x[p][0].x, x[p][1].x),
                                                   make_float2(x[p][2].x, x[p][3].x));
-                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.x) = he;
+                    f16_store(b4 + o.x, he);
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) =
                         quant_row4<FP8>(x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y, ip.y);
                 } else {
@@ -761,7 +775,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                         quant_row4<FP8>(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x, ip.x);
                     const uint2 ho = quant_fp16x4(make_float2(x[p][0].y, x[p][1].y),
                                                   make_float2(x[p][2].y, x[p][3].y));
-                    *reinterpret_cast<uint2*>(const_cast<uint8_t*>(b8) + o.y) = ho;
+                    f16_store(b4 + o.y, ho);
                 }
             }
             fence_proxy_async_smem();

@@ -149,10 +149,10 @@ __device__ __forceinline__ void row_formats(uint4 mask, int r0, uint32_t& bits, 
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
-// Two FP32 products, each rounded to nearest even.  Written as two scalar
-// multiplies: on sm_100a the packed f32x2 multiply did not reproduce the
-// scalar round-to-nearest product for every operand pair, and every product
-// here feeds a stored, bit-exact value.
+// Two FP32 products, each rounded to nearest even, as two scalar multiplies.
+// (The d = 128 kernel forms the same products with the packed f32x2
+// multiply, which rounds each half the same way; its states are checked
+// bit for bit against these kernels and the oracle.)
 __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
     return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
 }
@@ -274,8 +274,10 @@ __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off,
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         if ((bits >> i) & 1u) {
-            *reinterpret_cast<uint2*>(blk + f16_off + (size_t)r16 * (2 * D) + cg * 8) =
-                quant_fp16x4(x[i][0], x[i][1]);
+            const uint2 h = quant_fp16x4(x[i][0], x[i][1]);
+            uint8_t* row = blk + f16_off + (size_t)r16 * (2 * D);
+            *reinterpret_cast<uint32_t*>(row + cg * 4) = h.x;
+            *reinterpret_cast<uint32_t*>(row + D + cg * 4) = h.y;
             ++r16;
         } else {
             *reinterpret_cast<uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4) =
@@ -291,9 +293,9 @@ __device__ __forceinline__ void store_quant_tile(uint8_t* blk, uint32_t f16_off,
 // Shared-memory variants for the decode step, addressed through the head's
 // row directory (one word per key row: row offset, scale offset, FP16 flag).
 // The block sits in a pipeline stage followed by at least 256 more bytes of
-// the same allocation, so both candidate reads of a row (8 bytes as FP16, 4
-// bytes as INT8, plus the scale) are always in bounds and can be issued
-// unconditionally: no load waits on a branch, and the rows' dependency chains
+// the same allocation, so both candidate reads of a row (the FP16 row's two
+// plane words, the byte row's word, which is the first of them, and the
+// scale) are always in bounds and can be issued unconditionally: no load waits on a branch, and the rows' dependency chains
 // overlap.  Stores are made per the row's format.
 // ---------------------------------------------------------------------------
 
@@ -332,7 +334,8 @@ __device__ __forceinline__ void load_tile_gdir(const uint8_t* blk, const uint32_
     for (int i = 0; i < RPT; ++i) {
         const uint8_t* row = blk + dir_row(e[i]);
         if (e[i] >> 31) {
-            raw[i] = __ldg(reinterpret_cast<const uint2*>(row + cg * 8));
+            raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(row + cg * 4));
+            raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(row + D + cg * 4));
         } else {
             raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(row + cg * 4));
             raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(blk + dir_scale(e[i])));
@@ -368,8 +371,8 @@ __device__ __forceinline__ void load_tile_dir(const uint8_t* blk, const uint32_t
         for (int j = 0; j < BATCH; ++j) {
             e[j] = dir[r0 + i0 + j];
             const uint8_t* row = blk + dir_row(e[j]);
-            w16[j] = *reinterpret_cast<const uint2*>(row + cg * 8);
             w8[j] = *reinterpret_cast<const uint32_t*>(row + cg * 4);
+            w16[j] = make_uint2(w8[j], *reinterpret_cast<const uint32_t*>(row + D + cg * 4));
             sc[j] = *reinterpret_cast<const float*>(blk + dir_scale(e[j]));
         }
 #pragma unroll
@@ -409,7 +412,9 @@ __device__ __forceinline__ void store_tile_dir(uint8_t* blk, const uint32_t* dir
         const uint32_t e = dir[r0 + i];
         uint8_t* row = blk + dir_row(e);
         if (e >> 31) {
-            *reinterpret_cast<uint2*>(row + cg * 8) = quant_fp16x4(x[i][0], x[i][1]);
+            const uint2 h = quant_fp16x4(x[i][0], x[i][1]);
+            *reinterpret_cast<uint32_t*>(row + cg * 4) = h.x;
+            *reinterpret_cast<uint32_t*>(row + D + cg * 4) = h.y;
         } else {
             *reinterpret_cast<uint32_t*>(row + cg * 4) =
                 FP8 ? quant_e4m3x4(x[i][0], x[i][1], rowbuf[RPT + i])

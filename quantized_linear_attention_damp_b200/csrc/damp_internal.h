@@ -30,6 +30,15 @@ __host__ __device__ inline uint32_t dir_scale(uint32_t e) { return (e >> 16) & 0
 __host__ __device__ inline uint32_t dir_entry(uint32_t row_off, uint32_t scale_off, bool f16) {
     return row_off | ((scale_off >> 2) << 18) | (f16 ? 0x80000000u : 0u);
 }
+// An FP16 row of d_v values is stored as two planes of d_v bytes: values 4g
+// and 4g + 1 of column group g in the first plane at byte 4g, values 4g + 2
+// and 4g + 3 in the second at d_v + 4g.  A thread holding the 4 columns of
+// group g then reads an FP16 row with the same 4-byte stride as a byte row
+// (one word in each plane, the byte row's word at the same offset as the
+// first).  Byte offset of value j:
+__host__ __device__ inline uint32_t f16_pos(uint32_t j, uint32_t d_v) {
+    return ((j >> 1) & 1u) * d_v + 4u * (j >> 2) + 2u * (j & 1u);
+}
 inline size_t dir_offset(int H) { return (kStatusBytes + (size_t)H * kMaskWords * 4 + 15) / 16 * 16; }
 inline size_t head_table_offset(int H, int d_k) { return dir_offset(H) + (size_t)H * d_k * 4; }
 

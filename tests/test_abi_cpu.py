@@ -190,12 +190,17 @@ def test_block_logical_round_trip(d, dv, hp):
             assert np.array_equal(back["scale"], scale)
             assert np.array_equal(back["half"], half)
             assert np.array_equal(back["code"], code)
-            # byte order: scales of INT8 rows first, then FP16 rows, then INT8 rows
+            # byte order: scales of INT8 rows first, then FP16 rows, then INT8 rows;
+            # an FP16 row is two planes: values 4g, 4g+1 of each column group g,
+            # then values 4g+2, 4g+3
             r = d - hp
             assert np.array_equal(raw[:4 * r].view(np.float32), scale[~is16])
             f16_off = (4 * r + 15) // 16 * 16
+            groups = half[is16].reshape(hp, dv // 4, 4)
+            planes = np.concatenate([groups[:, :, 0:2].reshape(hp, dv // 2),
+                                     groups[:, :, 2:4].reshape(hp, dv // 2)], axis=1)
             assert np.array_equal(raw[f16_off:f16_off + 2 * hp * dv].view(np.uint16),
-                                  half[is16].reshape(-1))
+                                  planes.reshape(-1))
             assert np.array_equal(raw[f16_off + 2 * hp * dv:f16_off + 2 * hp * dv + r * dv]
                                   .view(np.int8), code[~is16].reshape(-1))
     finally:
