@@ -275,27 +275,51 @@ class Bench:
 
     def timed_e2e(self, steps: int) -> tuple[float, int, int]:
         """Same steps through the public API from pinned host memory: each step
-        copies its inputs H2D, runs, and copies out D2H (device-timed)."""
+        copies its inputs H2D, runs, and copies `out` D2H (device-timed, one
+        event pair around all steps).  As a serving loop would, the copies run
+        on their own streams, double-buffered, so that step i's kernel overlaps
+        the input copy of step i+1 and the output copy of step i-1."""
         torch = self.torch
-        dev_in = {k: torch.empty_like(v, device=self.dev) for k, v in self.host[0].items()}
-        out_host = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        dev_in = [{k: torch.empty_like(v, device=self.dev) for k, v in self.host[0].items()}
+                  for _ in range(2)]
+        outs = [torch.empty_like(self.out) for _ in range(2)]
+        out_host = [torch.empty(self.out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in self.host[0].values())
-        d2h = out_host.numel() * 4
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(steps)]
+        d2h = out_host[0].numel() * 4
+        comp = torch.cuda.current_stream(self.dev)
+        s_in, s_out = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
+        ev = lambda: torch.cuda.Event()
+        copied = [ev() for _ in range(steps)]    # inputs of step i on the device
+        ran = [ev() for _ in range(steps)]       # kernel of step i done
+        read = [ev() for _ in range(steps)]      # out of step i on the host
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize(self.dev)
+        e0.record(comp)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
         for i in range(steps):
-            src = self.host[i % len(self.host)]
-            ev[i][0].record()
-            for k_, v_ in src.items():
-                dev_in[k_].copy_(v_, non_blocking=True)
-            self.pools[i % self.n_pools].step(dev_in["slot_idx"], dev_in["q"], dev_in["k"],
-                                              dev_in["v"], dev_in["alpha"], dev_in["beta"],
-                                              self.out)
-            out_host.copy_(self.out, non_blocking=True)
-            ev[i][1].record()
+            src, buf, o = self.host[i % len(self.host)], dev_in[i % 2], outs[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ran[i - 2])          # buffer free again
+                for k_, v_ in src.items():
+                    buf[k_].copy_(v_, non_blocking=True)
+                copied[i].record(s_in)
+            comp.wait_event(copied[i])
+            if i >= 2:
+                comp.wait_event(read[i - 2])             # out buffer read back
+            self.pools[i % self.n_pools].step(buf["slot_idx"], buf["q"], buf["k"], buf["v"],
+                                              buf["alpha"], buf["beta"], o, stream=comp)
+            ran[i].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ran[i])
+                out_host[i % 2].copy_(o, non_blocking=True)
+                read[i].record(s_out)
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
+        e1.record(comp)
         torch.cuda.synchronize(self.dev)
-        return sum(a.elapsed_time(b) for a, b in ev) / 1e3, h2d, d2h
+        return e0.elapsed_time(e1) / 1e3, h2d, d2h
 
     def close(self):
         for p in self.pools:
