@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kCodecThreads) codec_kernel(const CodecArgs a)
                 continue;
             }
             if constexpr (QUANT) {
-                load_tile_gdir<D, FP8>(blk, a.dir + (size_t)h * D, r0, cg, x);
+                load_tile_mask<D, FP8>(blk, hb.z, hb.w, bits, rank16, r0, cg, x);
             } else {
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {

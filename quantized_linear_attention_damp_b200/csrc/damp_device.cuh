@@ -319,31 +319,32 @@ __device__ __forceinline__ void dequant_int8x4_packed(uint32_t w, float s, float
 }
 
 // Rows [r0, r0+RPT) x cols [4cg, 4cg+4) of a quantized block in global memory,
-// addressed through the head's row directory.  Every row's loads are issued
-// before the first is used, so a thread's reads overlap instead of waiting one
-// after another behind the format branches.
+// located from the row-format bits of the thread's rows (bit i: row r0 + i is
+// FP16) and rank16 (FP16 rows below r0), as store_quant_tile does: no load
+// waits on another, so every row's reads are in flight together.
 template <int D, bool FP8 = false>
-__device__ __forceinline__ void load_tile_gdir(const uint8_t* blk, const uint32_t* dir, int r0,
-                                               int cg, float2 (&x)[Geo<D>::RPT][2]) {
+__device__ __forceinline__ void load_tile_mask(const uint8_t* blk, uint32_t f16_off, uint32_t i8_off,
+                                               uint32_t bits, int rank16, int r0, int cg,
+                                               float2 (&x)[Geo<D>::RPT][2]) {
     constexpr int RPT = Geo<D>::RPT;
-    uint32_t e[RPT];
-    uint2 raw[RPT];   // FP16 row: 4 values; byte row: 4 codes in .x, the row's scale in .y
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) e[i] = __ldg(dir + r0 + i);
+    uint2 raw[RPT];   // FP16 row: its two plane words; byte row: 4 codes in .x, the row's scale in .y
+    int r16 = rank16, r8 = r0 - rank16;
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-        const uint8_t* row = blk + dir_row(e[i]);
-        if (e[i] >> 31) {
+        if ((bits >> i) & 1u) {
+            const uint8_t* row = blk + f16_off + (size_t)r16 * (2 * D);
             raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(row + cg * 4));
             raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(row + D + cg * 4));
+            ++r16;
         } else {
-            raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(row + cg * 4));
-            raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(blk + dir_scale(e[i])));
+            raw[i].x = __ldg(reinterpret_cast<const uint32_t*>(blk + i8_off + (size_t)r8 * D + cg * 4));
+            raw[i].y = __ldg(reinterpret_cast<const uint32_t*>(blk + (size_t)r8 * 4));
+            ++r8;
         }
     }
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-        if (e[i] >> 31) dequant_fp16x4(raw[i], x[i][0], x[i][1]);
+        if ((bits >> i) & 1u) dequant_fp16x4(raw[i], x[i][0], x[i][1]);
         else if constexpr (FP8) dequant_e4m3x4(raw[i].x, __uint_as_float(raw[i].y), x[i][0], x[i][1]);
         else dequant_int8x4_packed(raw[i].x, __uint_as_float(raw[i].y), x[i][0], x[i][1]);
     }
