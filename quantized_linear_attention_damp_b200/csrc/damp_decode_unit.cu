@@ -95,13 +95,6 @@ __device__ __forceinline__ float in_at(const uint8_t* base, int idx) {
     }
 }
 
-// INT8 code c (byte c of w, two's complement) as the float 2^23 + 128 + code,
-// exactly: wb = w ^ 0x80808080 holds the codes biased to 1..255, and the byte
-// permute places one of them in the low mantissa bits of 2^23.
-__device__ __forceinline__ float i8_biased(uint32_t wb, int c) {
-    return __uint_as_float(__byte_perm(wb, 0x4B000000u, 0x7440u | (uint32_t)c));
-}
-
 // The four E4M3 codes of w widened exactly to FP32 (E4M3 is a subset of FP16).
 __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
     uint32_t h01, h23;
@@ -110,25 +103,6 @@ __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&f)[4]) {
     const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h01));
     const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h23));
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-}
-
-__device__ __forceinline__ void f16x4_to_f32(uint2 h, float (&f)[4]) {
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-}
-
-// Values of one byte row (4 codes) before the scale: INT8 -> 2^23 + 128 + code
-// (the bias is removed by the caller), FP8 -> the E4M3 value.
-template <bool FP8>
-__device__ __forceinline__ void byte_row_raw(uint32_t w, float (&f)[4]) {
-    if constexpr (FP8) {
-        e4m3x4_to_f32(w, f);
-    } else {
-        const uint32_t wb = w ^ 0x80808080u;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) f[c] = i8_biased(wb, c);
-    }
 }
 
 // A float2 held in one 64-bit register (the operand type of the packed FP32
@@ -151,8 +125,8 @@ __device__ __forceinline__ unsigned long long as_u64(float2 v) {
 // first word).  Each row's format is a uniform branch (bra.uni: the same in
 // every lane); the offset and the scale are packed operations on the pair.
 __device__ __forceinline__ void pair_decode(int P, uint32_t m, uint32_t we0, uint32_t we1,
-                                                uint32_t wo0, uint32_t wo1, float2 bz, float2 sp,
-                                                float2 (&x)[4]) {
+                                            uint32_t wo0, uint32_t wo1, float2 bz, float2 sp,
+                                            float2 (&x)[4]) {
     unsigned long long r0, r1, r2, r3;
     asm("{\n\t"
         ".reg .pred p, pe, po;\n\t"
@@ -257,28 +231,9 @@ __device__ __forceinline__ void pair_store(int P, uint32_t m, uint32_t ae, uint3
         : "memory");
 }
 
-// This lane's two words of an FP16 row (one per plane) and their store.
-__device__ __forceinline__ uint2 f16_words(const uint8_t* w) {
-    return make_uint2(*reinterpret_cast<const uint32_t*>(w), *reinterpret_cast<const uint32_t*>(w + kPD));
-}
-__device__ __forceinline__ void f16_store(const uint8_t* w, uint2 h) {
-    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(w)) = h.x;
-    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(w) + kPD) = h.y;
-}
-
 // max |v| over 4 values
 __device__ __forceinline__ float absmax4v(float a, float b, float c, float d) {
     return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
-}
-
-// Codes of one byte row (4 values, row inverse scale inv), packed in a word.
-template <bool FP8>
-__device__ __forceinline__ uint32_t quant_row4(float a, float b, float c, float d, float inv) {
-    if constexpr (FP8) {
-        return quant_e4m3x4(make_float2(a, b), make_float2(c, d), inv);
-    } else {
-        return quant_int8x4(make_float2(a, b), make_float2(c, d), inv);
-    }
 }
 
 // Two byte rows at once (inverse scales as a pair).
@@ -287,7 +242,7 @@ __device__ __forceinline__ uint2 quant_pair4(const float2 (&x)[4], float2 inv) {
     if constexpr (FP8) {
         float2 y[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) y[c] = mul2_rn(x[c], inv);
+        for (int c = 0; c < 4; ++c) y[c] = __fmul2_rn(x[c], inv);
         unsigned short e01, e23, o01, o23;
         asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e01) : "f"(y[1].x), "f"(y[0].x));
         asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e23) : "f"(y[3].x), "f"(y[2].x));
@@ -503,7 +458,6 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             // ---- step 1 (reconstruct) and step 2 (first half), pair by pair:
             // S' = D S^; u = k^T S' (pairwise); w = q^T S'
             const float2 al_g = f2(meta.alpha);
-            const float2 bias2 = f2(-8388736.0f);   // -(2^23 + 128)
             float2 wacc[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) wacc[c] = f2(0.f);
@@ -511,7 +465,6 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             float2 usum[2];
 #pragma unroll
             for (int p = 0; p < kPP; ++p) {
-                const uint32_t fm = (m16 >> (2 * p)) & 3u;   // bit0: row 2p FP16; bit1: row 2p+1
                 const uint2 o = tab->off[p];
                 const float4 bs = tab->bs[p];
                 const float2 sp = make_float2(bs.z, bs.w);
@@ -524,41 +477,13 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     const uint32_t* pe = reinterpret_cast<const uint32_t*>(b4 + o.x);
                     const uint32_t* po = reinterpret_cast<const uint32_t*>(b4 + o.y);
                     pair_decode(p, m16, pe[0], pe[kPD / 4], po[0], po[kPD / 4], tab->bz[p], sp, x[p]);
-                } else if (fm == 0u) {
-                    float e[4], d[4];
-                    byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
-                    byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float2 t = make_float2(e[c], d[c]);
-                        if constexpr (!FP8) t = __fadd2_rn(t, bias2);
-                        x[p][c] = __fmul2_rn(t, sp);
-                    }
-                } else if (fm == 3u) {
-                    float e[4], d[4];
-                    f16x4_to_f32(f16_words(b4 + o.x), e);
-                    f16x4_to_f32(f16_words(b4 + o.y), d);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) x[p][c] = make_float2(e[c], d[c]);
                 } else {
-                    // one FP16 row and one byte row: the FP16 half is offset by
-                    // -0 and scaled by 1 (both exact, signed zeros kept)
+                    // FP8 pools hold no FP16 rows: both rows are E4M3 rows
                     float e[4], d[4];
-                    if (fm == 1u) {
-                        f16x4_to_f32(f16_words(b4 + o.x), e);
-                        byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
-                    } else {
-                        byte_row_raw<FP8>(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
-                        f16x4_to_f32(f16_words(b4 + o.y), d);
-                    }
-                    const float2 bz = fm == 1u ? make_float2(-0.0f, -8388736.0f)
-                                               : make_float2(-8388736.0f, -0.0f);
+                    e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(b4 + o.x), e);
+                    e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(b4 + o.y), d);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float2 t = make_float2(e[c], d[c]);
-                        if constexpr (!FP8) t = __fadd2_rn(t, bz);
-                        x[p][c] = __fmul2_rn(t, sp);
-                    }
+                    for (int c = 0; c < 4; ++c) x[p][c] = __fmul2_rn(make_float2(e[c], d[c]), sp);
                 }
                 const float2 alp = KDA ? tab->al[p] : al_g;
                 const float4 kq = tab->kq[p];
@@ -694,12 +619,10 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             float am[kRW];
 #pragma unroll
             for (int p = 0; p < kPP; ++p) {
-                const uint32_t fm = (m16 >> (2 * p)) & 3u;
                 const float4 bs = tab->bs[p];
                 const float2 bp = make_float2(bs.x, bs.y);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) x[p][c] = __ffma2_rn(bp, dl[c], x[p][c]);
-                (void)fm;
                 am[2 * p] = __uint_as_float(__reduce_max_sync(
                     0xffffffffu, __float_as_uint(absmax4v(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x))));
                 am[2 * p + 1] = __uint_as_float(__reduce_max_sync(
@@ -746,36 +669,17 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             __syncwarp();
 #pragma unroll
             for (int p = 0; p < kPP; ++p) {
-                const uint32_t fm = (m16 >> (2 * p)) & 3u;
                 const uint2 o = tab->off[p];
                 const float2 ip = *reinterpret_cast<const float2*>(&tab->inv[2 * p]);
                 if constexpr (!FP8) {
                     const uint2 cw = quant_pair4<false>(x[p], ip);
                     const uint32_t s4 = smem_u32(b4);
                     pair_store(p, m16, s4 + o.x, s4 + o.y, cw, x[p]);
-                } else if (fm == 0u) {
+                } else {
+                    // FP8 pools hold no FP16 rows: two E4M3 code words
                     const uint2 cw = quant_pair4<FP8>(x[p], ip);
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) = cw.x;
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) = cw.y;
-                } else if (fm == 3u) {
-                    const uint2 he = quant_fp16x4(make_float2(x[p][0].x, x[p][1].x),
-                                                  make_float2(x[p][2].x, x[p][3].x));
-                    const uint2 ho = quant_fp16x4(make_float2(x[p][0].y, x[p][1].y),
-                                                  make_float2(x[p][2].y, x[p][3].y));
-                    f16_store(b4 + o.x, he);
-                    f16_store(b4 + o.y, ho);
-                } else if (fm == 1u) {
-                    const uint2 he = quant_fp16x4(make_float2(x[p][0].x, x[p][1].x),
-                                                  make_float2(x[p][2].x, x[p][3].x));
-                    f16_store(b4 + o.x, he);
-                    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) =
-                        quant_row4<FP8>(x[p][0].y, x[p][1].y, x[p][2].y, x[p][3].y, ip.y);
-                } else {
-                    *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) =
-                        quant_row4<FP8>(x[p][0].x, x[p][1].x, x[p][2].x, x[p][3].x, ip.x);
-                    const uint2 ho = quant_fp16x4(make_float2(x[p][0].y, x[p][1].y),
-                                                  make_float2(x[p][2].y, x[p][3].y));
-                    f16_store(b4 + o.y, ho);
                 }
             }
             fence_proxy_async_smem();
