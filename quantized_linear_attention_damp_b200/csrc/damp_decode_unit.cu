@@ -60,6 +60,9 @@ constexpr int kRW = 16;        // key rows per warp
 constexpr int kPP = kRW / 2;   // row pairs per warp
 constexpr int kNW = kPT / 32;  // warps
 constexpr uint32_t kDirBytes = kPD * 4;   // the head's row directory
+// Row formats of a pool: FP16 and INT8 rows (per the directory), INT8 rows
+// only, or E4M3 rows only (no format test per row in the last two).
+constexpr int kRowsMixed = 0, kRowsInt8 = 1, kRowsFp8 = 2;
 
 // Per-unit metadata written by the refill warp into the stage (32 bytes).
 struct PMeta {
@@ -185,6 +188,43 @@ __device__ __forceinline__ void pair_decode(int P, uint32_t m, uint32_t we0, uin
     x[0] = as_f2(r0); x[1] = as_f2(r1); x[2] = as_f2(r2); x[3] = as_f2(r3);
 }
 
+// Two byte rows of a pair decoded and dequantized (pools with no FP16 rows):
+// x[c] = fl((2^23 + 128 + code_c - (2^23 + 128)) * s) for row 2p (.x, codes
+// in we) and row 2p + 1 (.y, codes in wo).
+__device__ __forceinline__ void pair_decode_i8(uint32_t we, uint32_t wo, float2 sp, float2 (&x)[4]) {
+    unsigned long long r0, r1, r2, r3;
+    asm("{\n\t"
+        ".reg .b32 wb, vb, e0, e1, e2, e3, d0, d1, d2, d3;\n\t"
+        ".reg .b64 bz;\n\t"
+        "xor.b32 wb, %4, 0x80808080;\n\t"
+        "xor.b32 vb, %5, 0x80808080;\n\t"
+        "prmt.b32 e0, wb, %6, 0x7440;\n\t"
+        "prmt.b32 e1, wb, %6, 0x7441;\n\t"
+        "prmt.b32 e2, wb, %6, 0x7442;\n\t"
+        "prmt.b32 e3, wb, %6, 0x7443;\n\t"
+        "prmt.b32 d0, vb, %6, 0x7440;\n\t"
+        "prmt.b32 d1, vb, %6, 0x7441;\n\t"
+        "prmt.b32 d2, vb, %6, 0x7442;\n\t"
+        "prmt.b32 d3, vb, %6, 0x7443;\n\t"
+        "mov.b64 %0, {e0, d0};\n\t"
+        "mov.b64 %1, {e1, d1};\n\t"
+        "mov.b64 %2, {e2, d2};\n\t"
+        "mov.b64 %3, {e3, d3};\n\t"
+        "mov.b64 bz, {%7, %7};\n\t"
+        "add.rn.f32x2 %0, %0, bz;\n\t"
+        "add.rn.f32x2 %1, %1, bz;\n\t"
+        "add.rn.f32x2 %2, %2, bz;\n\t"
+        "add.rn.f32x2 %3, %3, bz;\n\t"
+        "mul.rn.f32x2 %0, %0, %8;\n\t"
+        "mul.rn.f32x2 %1, %1, %8;\n\t"
+        "mul.rn.f32x2 %2, %2, %8;\n\t"
+        "mul.rn.f32x2 %3, %3, %8;\n\t"
+        "}"
+        : "=l"(r0), "=l"(r1), "=l"(r2), "=l"(r3)
+        : "r"(we), "r"(wo), "r"(0x4B000000u), "r"(0xCB000080u), "l"(as_u64(sp)));
+    x[0] = as_f2(r0); x[1] = as_f2(r1); x[2] = as_f2(r2); x[3] = as_f2(r3);
+}
+
 // Store both rows of a pair at their words a_e, a_o: the two code words when
 // both are byte rows (one uniform test), else row by row (byte row -> its
 // code word; FP16 row -> its four values rounded to binary16, one word in
@@ -266,8 +306,9 @@ __device__ __forceinline__ uint2 quant_pair4(const float2 (&x)[4], float2 inv) {
     }
 }
 
-template <bool KDA, bool BF16, bool FP8>
+template <bool KDA, bool BF16, int ROWS>
 __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
+    constexpr bool FP8 = ROWS == kRowsFp8, I8 = ROWS == kRowsInt8;
     constexpr uint32_t ELT = BF16 ? 2 : 4;
     constexpr float kQ = FP8 ? 448.0f : 127.0f;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -468,7 +509,11 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 const uint2 o = tab->off[p];
                 const float4 bs = tab->bs[p];
                 const float2 sp = make_float2(bs.z, bs.w);
-                if constexpr (!FP8) {
+                if constexpr (I8) {
+                    // INT8 pools hold no FP16 rows: both rows are INT8 rows
+                    pair_decode_i8(*reinterpret_cast<const uint32_t*>(b4 + o.x),
+                                   *reinterpret_cast<const uint32_t*>(b4 + o.y), sp, x[p]);
+                } else if constexpr (!FP8) {
                     // each row's words (a byte row's word, or an FP16 row's
                     // two plane words; a byte row also reads the word 128
                     // bytes on, inside the stage, and does not use it),
@@ -671,12 +716,12 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             for (int p = 0; p < kPP; ++p) {
                 const uint2 o = tab->off[p];
                 const float2 ip = *reinterpret_cast<const float2*>(&tab->inv[2 * p]);
-                if constexpr (!FP8) {
+                if constexpr (ROWS == kRowsMixed) {
                     const uint2 cw = quant_pair4<false>(x[p], ip);
                     const uint32_t s4 = smem_u32(b4);
                     pair_store(p, m16, s4 + o.x, s4 + o.y, cw, x[p]);
                 } else {
-                    // FP8 pools hold no FP16 rows: two E4M3 code words
+                    // INT8 or FP8 pools hold no FP16 rows: two code words
                     const uint2 cw = quant_pair4<FP8>(x[p], ip);
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.x) = cw.x;
                     *reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(b4) + o.y) = cw.y;
@@ -748,24 +793,24 @@ uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
 constexpr uint32_t kBudget1 = 227u * 1024u;
 constexpr uint32_t kBudget2 = 228u * 1024u / 2 - 1024u;
 
-template <bool KDA, bool BF16, bool FP8>
+template <bool KDA, bool BF16, int ROWS>
 cudaError_t unit_attrs_t() {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(decode_unit_kernel<KDA, BF16, FP8>,
+        attr_err = cudaFuncSetAttribute(decode_unit_kernel<KDA, BF16, ROWS>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(decode_unit_kernel<KDA, BF16, FP8>,
+            attr_err = cudaFuncSetAttribute(decode_unit_kernel<KDA, BF16, ROWS>,
                                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     });
     return attr_err;
 }
 
-template <bool KDA, bool BF16, bool FP8>
+template <bool KDA, bool BF16, int ROWS>
 cudaError_t launch_unit_t(const StepArgs& a0, cudaStream_t stream) {
-    auto kern = decode_unit_kernel<KDA, BF16, FP8>;
-    const cudaError_t attr_err = unit_attrs_t<KDA, BF16, FP8>();
+    auto kern = decode_unit_kernel<KDA, BF16, ROWS>;
+    const cudaError_t attr_err = unit_attrs_t<KDA, BF16, ROWS>();
     if (attr_err != cudaSuccess) return attr_err;
     StepArgs a = a0;
     int dev = 0, sms = 0;
@@ -803,16 +848,20 @@ cudaError_t launch_unit_t(const StepArgs& a0, cudaStream_t stream) {
 
 }  // namespace
 
+template <int ROWS>
+cudaError_t prepare_rows() {
+    cudaError_t e;
+    if ((e = unit_attrs_t<false, false, ROWS>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<false, true, ROWS>()) != cudaSuccess) return e;
+    if ((e = unit_attrs_t<true, false, ROWS>()) != cudaSuccess) return e;
+    return unit_attrs_t<true, true, ROWS>();
+}
+
 cudaError_t prepare_decode_unit() {
     cudaError_t e;
-    if ((e = unit_attrs_t<false, false, false>()) != cudaSuccess) return e;
-    if ((e = unit_attrs_t<false, true, false>()) != cudaSuccess) return e;
-    if ((e = unit_attrs_t<true, false, false>()) != cudaSuccess) return e;
-    if ((e = unit_attrs_t<true, true, false>()) != cudaSuccess) return e;
-    if ((e = unit_attrs_t<false, false, true>()) != cudaSuccess) return e;
-    if ((e = unit_attrs_t<false, true, true>()) != cudaSuccess) return e;
-    if ((e = unit_attrs_t<true, false, true>()) != cudaSuccess) return e;
-    return unit_attrs_t<true, true, true>();
+    if ((e = prepare_rows<kRowsMixed>()) != cudaSuccess) return e;
+    if ((e = prepare_rows<kRowsInt8>()) != cudaSuccess) return e;
+    return prepare_rows<kRowsFp8>();
 }
 
 bool decode_unit_fits(const StepArgs& a, int in_dtype, int gate) {
@@ -820,18 +869,18 @@ bool decode_unit_fits(const StepArgs& a, int in_dtype, int gate) {
     return unit_layout(b, gate == DAMP_GATE_VECTOR, in_dtype == DAMP_DTYPE_BF16, kBudget1) != 0;
 }
 
+template <int ROWS>
+cudaError_t launch_rows(const StepArgs& a, bool kda, bool bf, cudaStream_t stream) {
+    if (kda) return bf ? launch_unit_t<true, true, ROWS>(a, stream) : launch_unit_t<true, false, ROWS>(a, stream);
+    return bf ? launch_unit_t<false, true, ROWS>(a, stream) : launch_unit_t<false, false, ROWS>(a, stream);
+}
+
 cudaError_t launch_decode_unit(const StepArgs& a, int in_dtype, int gate, bool fp8,
                                cudaStream_t stream) {
     const bool kda = gate == DAMP_GATE_VECTOR, bf = in_dtype == DAMP_DTYPE_BF16;
-    if (fp8) {
-        if (kda)
-            return bf ? launch_unit_t<true, true, true>(a, stream)
-                      : launch_unit_t<true, false, true>(a, stream);
-        return bf ? launch_unit_t<false, true, true>(a, stream)
-                  : launch_unit_t<false, false, true>(a, stream);
-    }
-    if (kda) return bf ? launch_unit_t<true, true, false>(a, stream) : launch_unit_t<true, false, false>(a, stream);
-    return bf ? launch_unit_t<false, true, false>(a, stream) : launch_unit_t<false, false, false>(a, stream);
+    if (fp8) return launch_rows<kRowsFp8>(a, kda, bf, stream);
+    if (a.format == DAMP_FMT_INT8_ROW) return launch_rows<kRowsInt8>(a, kda, bf, stream);
+    return launch_rows<kRowsMixed>(a, kda, bf, stream);
 }
 
 }  // namespace damp
