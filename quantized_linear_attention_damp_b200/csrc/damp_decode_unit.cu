@@ -25,7 +25,9 @@
 // branch, so that the loads of later rows can be issued ahead; the decode,
 // and later the store, are inline PTX with a branch on the row's format
 // marked bra.uni: the format is the same in every lane, so the branch needs
-// no reconvergence.  A pair of byte rows is stored behind one test.
+// no reconvergence.  A pair of byte rows is stored behind one test.  Pools
+// of INT8 rows only or E4M3 rows only have their own instantiation, with no
+// format test at all.
 //
 // Two CTAs share an SM whenever three stages fit in half of its shared
 // memory (4 stages at 27 FP16 rows): their barriers are independent, so one
@@ -40,7 +42,10 @@
 // decays and the head's row directory into a shared-memory ring of stages
 // completing on mbarriers; no tensor map, no multicast).  A named barrier
 // between the two lets the refill start as soon as the stage's old store has
-// read it.
+// read it.  The refill sits on every item's critical path (the next barrier
+// waits for warp 7), so it is kept short: each lane of warp 7 holds the
+// metadata of every 32nd unit, loaded 32 units ahead with a division-free
+// cursor, and the lane that holds an item issues its copies itself.
 
 #include <cuda_runtime.h>
 
@@ -340,17 +345,29 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
         int head;
         uint2 hb;          // the head's {block offset in the slot, block size}
     };
+    // Lane L of the refill warp loads the units U = L, L + 32, L + 64, ... of
+    // this CTA (unit u = blockIdx + U * gridDim = b * H + h): it keeps (u, b, h)
+    // of its next unit and advances them by 32 * gridDim units each time, so
+    // no load needs a division.
+    const int du = 32 * (int)gridDim.x, db = du / H, dh = du - db * H;
+    int nu = (int)blockIdx.x + lane * (int)gridDim.x;
+    int nb = nu / H, nh = nu - nb * H;
     auto load_meta = [&](int U) {
         RMeta r{INT_MIN, 0.f, 0.f, -1, 0, make_uint2(0u, 0u)};
         if (U < my_items) {
-            const int u = (int)blockIdx.x + U * (int)gridDim.x;   // unit b*H + h
-            const int b = u / H, h = u - b * H;
-            r.head = h;
-            r.slot = __ldg(a.slot_idx + b);
-            r.unit = u;
-            if constexpr (!KDA) r.alpha = __ldg(a.alpha + u);
-            r.beta = __ldg(a.beta + u);
-            r.hb = __ldg(reinterpret_cast<const uint2*>(a.heads + h));
+            r.head = nh;
+            r.slot = __ldg(a.slot_idx + nb);
+            r.unit = nu;
+            if constexpr (!KDA) r.alpha = __ldg(a.alpha + nu);
+            r.beta = __ldg(a.beta + nu);
+            r.hb = __ldg(reinterpret_cast<const uint2*>(a.heads + nh));
+        }
+        nu += du;
+        nb += db;
+        nh += dh;
+        if (nh >= H) {
+            nh -= H;
+            ++nb;
         }
         return r;
     };
@@ -386,33 +403,28 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     auto issue = [&](int il) {
         const int stage = il % NS;
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
-        const int src = il & 31;
-        RMeta r;
-        r.slot = __shfl_sync(0xffffffffu, ring.slot, src);
-        r.alpha = __shfl_sync(0xffffffffu, ring.alpha, src);
-        r.beta = __shfl_sync(0xffffffffu, ring.beta, src);
-        r.unit = __shfl_sync(0xffffffffu, ring.unit, src);
-        r.head = __shfl_sync(0xffffffffu, ring.head, src);
-        r.hb.x = __shfl_sync(0xffffffffu, ring.hb.x, src);
-        r.hb.y = __shfl_sync(0xffffffffu, ring.hb.y, src);
-        const PMeta m = finish_meta(r);
-        if (lane == src) ring = load_meta(il + 32);
-        if (lane == 0 && !(il == 0 && (a.hooks & kHookHoldFirstItem))) {
-            *reinterpret_cast<PMeta*>(st + a.st_meta) = m;
-            const uint32_t fb = full_bar(stage);
-            if (m.active == 1) {
-                mbar_arrive_expect_tx(fb, m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u) + kDirBytes);
-                bulk_g2s(smem_u32(st), a.blocks + m.boff, m.bytes, fb);
-                const size_t io = (size_t)m.unit * kPD * ELT;
-                bulk_g2s(smem_u32(st + a.st_q), static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
-                bulk_g2s(smem_u32(st + a.st_k), static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
-                bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
-                if constexpr (KDA)
-                    bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + (size_t)m.unit * kPD, kPD * 4, fb);
-                bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)r.head * kPD, kDirBytes, fb);
-            } else {
-                mbar_arrive(fb);
+        // the lane that holds the item's metadata issues it (no shuffles)
+        if (lane == (il & 31)) {
+            const PMeta m = finish_meta(ring);
+            const int head = ring.head;
+            if (!(il == 0 && (a.hooks & kHookHoldFirstItem))) {
+                *reinterpret_cast<PMeta*>(st + a.st_meta) = m;
+                const uint32_t fb = full_bar(stage);
+                if (m.active == 1) {
+                    mbar_arrive_expect_tx(fb, m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u) + kDirBytes);
+                    bulk_g2s(smem_u32(st), a.blocks + m.boff, m.bytes, fb);
+                    const size_t io = (size_t)m.unit * kPD * ELT;
+                    bulk_g2s(smem_u32(st + a.st_q), static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
+                    bulk_g2s(smem_u32(st + a.st_k), static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
+                    bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
+                    if constexpr (KDA)
+                        bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + (size_t)m.unit * kPD, kPD * 4, fb);
+                    bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)head * kPD, kDirBytes, fb);
+                } else {
+                    mbar_arrive(fb);
+                }
             }
+            ring = load_meta(il + 32);
         }
         __syncwarp();
     };
