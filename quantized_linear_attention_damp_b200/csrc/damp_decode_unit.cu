@@ -37,15 +37,17 @@
 // the partials are double-buffered by item parity, so a warp that starts
 // the next item cannot overwrite them while another still reads them).
 // Meanwhile warp 6 writes back the previous unit's block (one bulk store,
-// once the barrier has ordered every writer's fenced rows before it) and
-// warp 7 refills the pipeline (cp.async.bulk of the block, q, k, v, the KDA
-// decays and the head's row directory into a shared-memory ring of stages
-// completing on mbarriers; no tensor map, no multicast).  A named barrier
-// between the two lets the refill start as soon as the stage's old store has
-// read it.  The refill sits on every item's critical path (the next barrier
-// waits for warp 7), so it is kept short: each lane of warp 7 holds the
-// metadata of every 32nd unit, loaded 32 units ahead with a division-free
-// cursor, and the lane that holds an item issues its copies itself.
+// once the barrier has ordered every writer's fenced rows before it) and the
+// two warps refill the pipeline: cp.async.bulk copies into a shared-memory
+// ring of stages completing on mbarriers (no tensor map, no multicast), two
+// arrivals per stage: warp 7 copies the block and the head's row directory,
+// warp 6 the unit's q, k, v and KDA decays.  Warp 6 waits for the stage's old
+// store to have read it before it arrives at the item's barrier, so after
+// the barrier both may reuse it.  The refill sits on every item's critical
+// path (the next barrier waits for these warps), so it is kept short and
+// split between them: each lane of warp 7 holds the metadata of every 32nd
+// unit, loaded 32 units ahead with a division-free cursor, and the lane that
+// holds an item issues its copies itself; warp 6 needs only the unit index.
 
 #include <cuda_runtime.h>
 
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 1);
+        for (int s = 0; s < NS; ++s) mbar_init(full_bar(s), 2);
         fence_mbar_init();
     }
     __syncthreads();
@@ -411,14 +413,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 *reinterpret_cast<PMeta*>(st + a.st_meta) = m;
                 const uint32_t fb = full_bar(stage);
                 if (m.active == 1) {
-                    mbar_arrive_expect_tx(fb, m.bytes + 3u * kPD * ELT + (KDA ? 4u * kPD : 0u) + kDirBytes);
+                    mbar_arrive_expect_tx(fb, m.bytes + kDirBytes);
                     bulk_g2s(smem_u32(st), a.blocks + m.boff, m.bytes, fb);
-                    const size_t io = (size_t)m.unit * kPD * ELT;
-                    bulk_g2s(smem_u32(st + a.st_q), static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
-                    bulk_g2s(smem_u32(st + a.st_k), static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
-                    bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
-                    if constexpr (KDA)
-                        bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + (size_t)m.unit * kPD, kPD * 4, fb);
                     bulk_g2s(smem_u32(st + a.st_dir), a.dir + (size_t)head * kPD, kDirBytes, fb);
                 } else {
                     mbar_arrive(fb);
@@ -427,6 +423,21 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             ring = load_meta(il + 32);
         }
         __syncwarp();
+    };
+
+    // The inputs of item il (store warp, lane 0): q, k, v and the KDA decays
+    // of unit blockIdx + il * gridDim, the stage's second arrival.
+    auto issue_inputs = [&](int il) {
+        const int stage = il % NS;
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const uint32_t fb = full_bar(stage);
+        const size_t u = (size_t)blockIdx.x + (size_t)il * gridDim.x;
+        const size_t io = u * kPD * ELT;
+        mbar_arrive_expect_tx(fb, 3u * kPD * ELT + (KDA ? 4u * kPD : 0u));
+        bulk_g2s(smem_u32(st + a.st_q), static_cast<const uint8_t*>(a.q) + io, kPD * ELT, fb);
+        bulk_g2s(smem_u32(st + a.st_k), static_cast<const uint8_t*>(a.k) + io, kPD * ELT, fb);
+        bulk_g2s(smem_u32(st + a.st_v), static_cast<const uint8_t*>(a.v) + io, kPD * ELT, fb);
+        if constexpr (KDA) bulk_g2s(smem_u32(st + a.st_alpha), a.alpha + u * kPD, kPD * 4, fb);
     };
 
     // One bulk store of item j's block (store warp, lane 0).
@@ -441,6 +452,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     int issued = 0;   // items issued so far (meaningful in the refill warp)
     if (warp == kIssueWarp)
         for (; issued < ahead && issued < my_items; ++issued) issue(issued);
+    if (warp == kStoreWarp && lane == 0)
+        for (int il = 0; il < ahead && il < my_items; ++il) issue_inputs(il);
 
     // ---- consumers: warp w owns rows [16w, 16w + 16), lane l columns [4l, 4l + 4)
     uint8_t* scratch = smem + a.scratch_off;
@@ -576,22 +589,23 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                 make_float4(__fadd_rn(wacc[0].x, wacc[0].y), __fadd_rn(wacc[1].x, wacc[1].y),
                             __fadd_rn(wacc[2].x, wacc[2].y), __fadd_rn(wacc[3].x, wacc[3].y));
         }
+        // the store of item it-2 (issued a whole item ago) has read its stage
+        // before the store warp arrives at the barrier, so after it the refill
+        // warp may reuse that stage
+        if (warp == kStoreWarp && lane == 0) bulk_wait_read<0>();
         if (bar_red_or(0, kPT, ok ? 0 : 1)) {
             aborted = true;
             break;
         }
 
         // ---- write back item it-1 (its requantized rows were fenced by their
-        // writers before this barrier) and refill the stage of item it-2 once
-        // that item's store has read it: the store warp checks the read,
-        // releases the refill warp through named barrier 2, then stores.
+        // writers before this barrier) and refill the stage of item it-2.
         if (warp == kStoreWarp) {
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-            asm volatile("bar.arrive 2, 64;" ::: "memory");
-            if (lane == 0 && it >= 1) store_item(it - 1);
+            if (lane == 0) {
+                if (it + ahead < my_items) issue_inputs(it + ahead);
+                if (it >= 1) store_item(it - 1);
+            }
         } else if (warp == kIssueWarp) {
-            asm volatile("bar.sync 2, 64;" ::: "memory");
             if (it + ahead < my_items) {
                 issue(it + ahead);
                 issued = it + ahead + 1;
