@@ -35,6 +35,12 @@ SMALL = {
                               gate=W.GATE_GDN, in_dtype="bf16"),
     "d128_kda_f32": W.Workload("d128_kda_f32", n=9, n_slots=9, H=4, d=128, hp=27, steps=3,
                                gate=W.GATE_KDA, in_dtype="f32"),
+    # the other two (gate, input type) pairs of the d = 128 kernel, so that every
+    # instantiation (row formats x gate x input type) runs
+    "d128_kda_bf16": W.Workload("d128_kda_bf16", n=11, n_slots=12, H=3, d=128, hp=27, steps=3,
+                                gate=W.GATE_KDA, in_dtype="bf16"),
+    "d128_gdn_f32": W.Workload("d128_gdn_f32", n=10, n_slots=10, H=3, d=128, hp=27, steps=3,
+                               gate=W.GATE_GDN, in_dtype="f32"),
 }
 
 
@@ -369,3 +375,32 @@ def test_sharded_pools_match_one_pool(gate):
         whole.close()
         for p in shards:
             p.close()
+
+
+@pytest.mark.parametrize("fmt", ["mixed", "int8"])
+def test_back_to_back_steps_same_pool(fmt):
+    """Consecutive steps on one pool launched with no host synchronisation in
+    between (each launch a programmatic dependent of the previous one, which
+    reads the blocks the previous one writes): after all of them, the state and
+    every step's readout equal the oracle's, bit for bit and within tolerance.
+    The batches repeat slots from step to step, so each step depends on the
+    last one's write-back."""
+    w = W.Workload("b2b_d128", n=40, n_slots=44, H=4, d=128, hp=27, steps=6,
+                   gate=W.GATE_GDN, in_dtype="bf16")
+    p = Pair(w, fmt)
+    try:
+        xs = [W.step_inputs(w, s, p.hs) for s in range(w.steps)]
+        ts = [torch_inputs(w, x) for x in xs]
+        outs = [torch.empty((w.n, w.H, w.d_v), dtype=torch.float32, device="cuda")
+                for _ in range(w.steps)]
+        torch.cuda.synchronize()
+        for t, o in zip(ts, outs):
+            p.gpu.step(t["slot_idx"], t["q"], t["k"], t["v"], t["alpha"], t["beta"], o)
+        torch.cuda.synchronize()
+        for x, o in zip(xs, outs):
+            p.check_out(o.cpu().numpy(), p.oracle_step_full(x))
+        rep = p.check_state()
+        assert rep["exact"], rep
+        assert p.gpu.get_error() == 0
+    finally:
+        p.close()
