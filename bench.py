@@ -479,7 +479,8 @@ def variants(args, dev):
     res = []
     steps = max(20, min(args.steps, 200))
     for name, fmt in [("hiconc_gdn", "int8"), ("hiconc_gdn", "fp8"), ("hiconc_gdn", "fp32"),
-                      ("gdn_batch", "mixed"), ("gdn_batch", "int8"), ("gdn_batch", "fp32")]:
+                      ("gdn_batch", "mixed"), ("gdn_batch", "int8"), ("gdn_batch", "fp32"),
+                      ("d64_gdn", "mixed"), ("d256_gdn", "mixed")]:
         w = W.WORKLOADS[name]
         b = Bench(w, fmt, device=dev)
         secs = b.timed(steps, 3)

@@ -88,6 +88,12 @@ WORKLOADS = {
     # 256 slots x 32 heads: the batch >= 256, 32-head, d=128 point
     "gdn_256x32": Workload("gdn_256x32", n=256, n_slots=256, H=32, d=128, hp=27, steps=32,
                            gate=GATE_GDN, in_dtype="bf16"),
+    # other state sizes (context for the other kernels): d=64 (square thread-tile kernel) and
+    # d=256 (any-shape kernel), FP16 rows ~21 % of the key rows as at d=128
+    "d64_gdn": Workload("d64_gdn", n=1024, n_slots=1024, H=32, d=64, hp=13, steps=32,
+                        gate=GATE_GDN, in_dtype="bf16"),
+    "d256_gdn": Workload("d256_gdn", n=256, n_slots=256, H=8, d=256, hp=54, steps=32,
+                         gate=GATE_GDN, in_dtype="bf16"),
 }
 
 
