@@ -83,15 +83,23 @@ struct PMeta {
 static_assert(sizeof(PMeta) == 32, "PMeta layout");
 
 // Per-warp table of the warp's 16 rows, as pairs (rows 2p, 2p + 1).
+// The entries read only before the item's barrier (the decays and the
+// dequantization offsets) share their space with those written only after it
+// (the row maxima and inverse scales): a warp fills its table for the next
+// item only after its last read of this item's.
 struct RowTab {
     float4 kq[kPP];      // {k_2p, k_2p+1, q_2p, q_2p+1}
     float4 bs[kPP];      // {b_2p, b_2p+1, s_2p, s_2p+1}: b = beta*k; s = row scale (1 for FP16 rows)
     uint2 off[kPP];      // byte offsets of rows 2p, 2p+1 in the block
-    float2 al[kPP];      // KDA decays of rows 2p, 2p+1
-    float2 bz[kPP];      // dequantization offsets of rows 2p, 2p+1: -(2^23+128) byte rows, -0 FP16 rows
+    union {
+        float2 al[kPP];  // KDA decays of rows 2p, 2p+1 (phase A)
+        float inv[kRW];  // Q / amax (byte rows; 0 for zero rows) (requantization)
+    };
+    union {
+        float2 bz[kPP];  // dequantization offsets of rows 2p, 2p+1: -(2^23+128) byte rows, -0 FP16 rows (phase A)
+        float amax[kRW]; // row maxima of |X| (byte rows) (requantization)
+    };
     uint32_t soff[kRW];  // byte offset of each byte row's scale in the block
-    float amax[kRW];     // row maxima of |X| (byte rows)
-    float inv[kRW];      // Q / amax (byte rows; 0 for zero rows)
 };
 static_assert(sizeof(RowTab) % 16 == 0, "RowTab layout");
 
@@ -338,8 +346,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     // U == L (mod 32), loaded 32 units ahead of use.  The ring holds raw
     // values: nothing waits for the loads until the unit is issued, and no
     // branch depends on a freshly loaded slot index.
-    constexpr int kIssueWarp = kNW - 1;         // refill
-    constexpr int kStoreWarp = kIssueWarp - 1;  // write-back
+    constexpr int kIssueWarp = kNW - 1;         // refill: metadata, block, directory
+    constexpr int kStoreWarp = kIssueWarp - 1;  // write-back; refill: q, k, v, KDA decays
     struct RMeta {
         int slot;          // slot index; INT_MIN: no such unit
         float alpha, beta;
@@ -400,8 +408,10 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    // Refill the stage of item il: metadata, then one bulk copy per operand,
-    // all completing on the stage's mbarrier (lane 0 issues them).
+    // The refill warp's part of item il: the stage's metadata, the block and
+    // the head's row directory (bulk copies completing on the stage's
+    // mbarrier, issued by the lane that holds the item's metadata); q, k, v
+    // and the KDA decays come from the store warp (issue_inputs).
     auto issue = [&](int il) {
         const int stage = il % NS;
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
@@ -461,8 +471,8 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
     // per-warp partial sums, double-buffered by item parity: a warp may start
     // the next item while others still read this item's partials
     float* red_w = red_u + 2 * kNW * kPD;               // [2][8][128], by warp
-    float* cpart_s = red_w + 2 * kNW * kPD;             // [2][8], by warp
-    RowTab* tab = reinterpret_cast<RowTab*>(cpart_s + 16) + warp;
+    float* cprod = red_w + 2 * kNW * kPD;               // [2][128]: fl(q_i beta k_i) by row
+    RowTab* tab = reinterpret_cast<RowTab*>(cprod + 2 * kPD) + warp;
     const int row0 = warp * kRW;
 
     int it = 0, stage = 0;
@@ -490,7 +500,6 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
             // ---- per-row operands of this warp's 16 rows (lanes 0-15, one row each)
             {
                 bool f16 = false;
-                float cp = 0.f;
                 if (lane < kRW) {
                     const int r = row0 + lane;
                     const uint32_t e = sdir[r];
@@ -512,13 +521,10 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                         reinterpret_cast<float*>(&tab->al[p])[j] =
                             reinterpret_cast<const float*>(st + a.st_alpha)[r];
                     tab->soff[lane] = so;
-                    cp = __fmul_rn(qr, br);
+                    // this row's term of c = q^T (beta k), summed by the warp that writes out
+                    cprod[(it & 1) * kPD + r] = __fmul_rn(qr, br);
                 }
                 m16 = __ballot_sync(0xffffffffu, f16);
-                // c = q^T (beta k) over this warp's rows (any order)
-#pragma unroll
-                for (int off = 8; off >= 1; off >>= 1) cp += __shfl_xor_sync(0xffffffffu, cp, off);
-                if (lane == 0) cpart_s[(it & 1) * kNW + warp] = cp;
                 __syncwarp();
             }
             // ---- step 1 (reconstruct) and step 2 (first half), pair by pair:
@@ -651,9 +657,10 @@ __global__ void __launch_bounds__(kPT, 2) decode_unit_kernel(const StepArgs a) {
                     ww[0] = __fadd2_rn(ww[0], make_float2(b0.x, b0.y));
                     ww[1] = __fadd2_rn(ww[1], make_float2(b0.z, b0.w));
                 }
-                const float4 c4a = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[0];
-                const float4 c4b = reinterpret_cast<const float4*>(cpart_s + (it & 1) * kNW)[1];
-                const float c = ((c4a.x + c4a.y) + (c4a.z + c4a.w)) + ((c4b.x + c4b.y) + (c4b.z + c4b.w));
+                const float4 c4 = reinterpret_cast<const float4*>(cprod + (it & 1) * kPD)[lane];
+                float c = (c4.x + c4.y) + (c4.z + c4.w);   // c = q^T (beta k), any order
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
                 const float2 o01 = __ffma2_rn(f2(c), d01, ww[0]);
                 const float2 o23 = __ffma2_rn(f2(c), d23, ww[1]);
                 reinterpret_cast<float4*>(a.out + (size_t)meta.unit * kPD)[lane] =
@@ -804,7 +811,7 @@ uint32_t unit_layout(StepArgs& a, bool kda, bool bf16, uint32_t budget) {
     off += sizeof(PMeta);
     a.stage_bytes = up(off, 128);
     const uint32_t scratch =
-        up((4 * kNW * kPD + 16) * 4 + kNW * (uint32_t)sizeof(RowTab), 128);
+        up((4 * kNW * kPD + 2 * kPD) * 4 + kNW * (uint32_t)sizeof(RowTab), 128);
     uint32_t ns = (budget - scratch - 128) / a.stage_bytes;
     if (ns > 6) ns = 6;
     if (ns < 3) return 0;
