@@ -79,7 +79,6 @@ __global__ void __launch_bounds__(kAnyThreads) decode_any_kernel(const StepArgs 
     __shared__ AnyRows R;
     __shared__ float s_delta[kMaxDim];
     __shared__ float s_c[kAnyWarps];
-    __shared__ int s_bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int d_k = a.d_k, d_v = a.d_v;
     const long long u = blockIdx.x;   // unit b*H + h
@@ -98,7 +97,6 @@ __global__ void __launch_bounds__(kAnyThreads) decode_any_kernel(const StepArgs 
 
     // ---- per-row operands and the pairwise merge schedule of d_k leaves
     if (tid == 0) {
-        s_bad = 0;
         for (int i = 0; i < d_k; ++i) R.merges[i] = 0;
         // internal node (lo, n) of the halving tree: its sum is formed right
         // after its last leaf lo + n - 1 (explicit stack of ranges)
